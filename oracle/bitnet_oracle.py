@@ -1,0 +1,304 @@
+"""CPU oracle of the BitNet b1.58 BitLinear forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its ``cpu_baseline``
+leg and its ``--impl reference`` arm) may import this module.  The product path
+(``ternary_bitlinear_quantized_b200``) never imports, calls or links it, and this
+module imports nothing from the product path.
+
+Plain numpy, written for reading, not speed.  Every quantity that decides an integer
+(a weight code, an int8 activation) is taken in fp32, the precision the CUDA kernels
+take it in; the exact sums that feed those decisions are integer (fixed-point) sums,
+so their result does not depend on the order of summation.  A library matmul serves
+as the integer dot product: it runs in fp64 on integer operands whose every partial
+sum stays below 2**53, so its result is exact.
+
+What each function follows (pages by title):
+
+* "Add optional RMSNorm support to BitNet quantization (config + layers)"
+  (transformers pull request): ``use_rms_norm`` / ``rms_norm_eps`` (default 1e-6);
+  BitLinear applies BitNetRMSNorm to the activations before quantising them;
+  ``BitNetMLP.forward`` = down(ffn_sub_norm(act(gate(x)) * up(x))).
+* "fix: I2_S ARM kernel layout + squared-ReLU FFN - passes the gate on the official
+  2B4T GGUF" (cpp-bitnet pull request), description bullets "I2_S NEON kernel for the
+  canonical layout" and "llama-quantize I2_S emits the canonical layout": 2-bit codes
+  c = w + 1 whose dot product is corrected by the activation sum; the interleaved
+  128-weight / 32-byte block layout; one scale per tensor stored after the packed data;
+  the zeroed trailer; rows divisible by 128; relu2 vs SiLU chosen from config.
+* BitNet b1.58 quantisers (absmean ternary weights, per-token absmax int8 activations),
+  as named by both pages above and by "More BitNet-like IQ1_S quantizations"
+  (llama.cpp discussion: 8-bit activations, ternary weights).
+
+Readings where the pages are silent (each also listed in the design doc):
+
+* bit order inside an I2_S block: element 128 b + 32 g + i is byte 32 b + i, bits
+  (7 - 2g):(6 - 2g) -- the interleaved layout, as opposed to the "sequential (byte
+  i/4, field i%4)" order the cpp-bitnet page calls wrong;
+* trailer: fp32 scale beta (little endian) then 28 zero bytes (32 bytes in all);
+* round() is round-half-to-even;
+* mean(x^2) and mean|W| are exact fixed-point sums (``fixed_point_mean_f32``) rounded
+  once to fp32; everything after them is a sequence of single IEEE fp32 operations;
+* the dequantisation factor is beta / s_x (= 1 / (s_x * s_w)) rounded to fp32, then
+  out = fp32(acc) * factor;
+* SiLU's exp is the fp64 ``pinned_exp`` below.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py`` (golden bytes,
+closed forms, invariants, brute force).  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import decimal
+import math
+
+import numpy as np
+
+F32 = np.float32
+F64 = np.float64
+QBLOCK = 128          # weights per I2_S block
+QBLOCK_BYTES = 32     # bytes per I2_S block
+TRAILER_BYTES = 32    # fp32 scale + 28 zero bytes
+ABS_FLOOR = F32(1e-5)  # the 1e-5 floor of both absmax and absmean
+
+
+# ----------------------------------------------------------------------------- sums
+
+def fixed_point_sum(terms: np.ndarray) -> tuple[int, int]:
+    """Order-free sum of non-negative fp64 ``terms`` on a fixed-point grid.
+
+    With M = max(terms) = m 2**E (0.5 <= m < 1) and 2**L >= n, the grid step is
+    2**-e with e = 62 - E - L: every term is below 2**(62 - L), so n of them sum below
+    2**62 in int64.  Each term is scaled by 2**e (exact) and rounded half-to-even to an
+    integer; the integer sum S is the same in any order.  Returns (S, e).
+    """
+    terms = np.asarray(terms, dtype=F64).ravel()
+    n = terms.size
+    if n == 0:
+        return 0, 0
+    M = float(terms.max())
+    if M == 0.0:
+        return 0, 0
+    _, E = math.frexp(M)
+    L = (n - 1).bit_length()
+    e = 62 - E - L
+    ints = np.rint(np.ldexp(terms, e)).astype(np.int64)
+    return int(ints.sum(dtype=np.int64)), e
+
+
+def fixed_point_mean_f32(terms: np.ndarray) -> np.float32:
+    """fp32( (fp64(S) * 2**-e) / n ): the mean of ``terms`` from ``fixed_point_sum``."""
+    terms = np.asarray(terms, dtype=F64).ravel()
+    S, e = fixed_point_sum(terms)
+    if S == 0:
+        return F32(0.0)
+    return F32(math.ldexp(float(S), -e) / float(terms.size))
+
+
+# ----------------------------------------------------------------------------- bf16
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) to fp32 exactly."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(F32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16, to nearest, ties to even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=F32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(f32_to_bf16_bits(x))
+
+
+# ----------------------------------------------------------------------------- a1: pack
+
+def i2s_packed_bytes(N: int, K: int) -> int:
+    """N*K/4 bytes of 2-bit codes, then the 32-byte trailer."""
+    return N * K // 4 + TRAILER_BYTES
+
+
+def absmean_scale(W: np.ndarray) -> np.float32:
+    """beta = max(mean|W|, 1e-5): the per-tensor weight scale (s_w = 1 / beta)."""
+    return np.maximum(fixed_point_mean_f32(np.abs(np.asarray(W, dtype=F32)).astype(F64)), ABS_FLOOR)
+
+
+def ternary_codes(W: np.ndarray, beta: np.float32) -> np.ndarray:
+    """c = clamp(round(W * s_w), -1, 1) + 1 with s_w = 1 / beta, in fp32."""
+    s_w = F32(1.0) / F32(beta)
+    w = np.asarray(W, dtype=F32) * s_w
+    return (np.clip(np.rint(w), -1, 1) + 1).astype(np.uint8)
+
+
+def interleave_i2s(codes: np.ndarray) -> np.ndarray:
+    """Codes [N, K] (values 0..2) -> N*K/4 bytes in the interleaved 128/32 layout."""
+    N, K = codes.shape
+    blk = codes.reshape(N * K // QBLOCK, 4, QBLOCK_BYTES).astype(np.uint8)  # [b, g, i]
+    out = (blk[:, 0, :] << 6) | (blk[:, 1, :] << 4) | (blk[:, 2, :] << 2) | blk[:, 3, :]
+    return out.reshape(-1).astype(np.uint8)
+
+
+def pack_i2s(W: np.ndarray) -> np.ndarray:
+    """Latent fp32 weights [N, K] -> I2_S bytes [N*K/4 + 32] (codes, fp32 beta, 28 zeros)."""
+    W = np.asarray(W, dtype=F32)
+    N, K = W.shape
+    if K % QBLOCK != 0:
+        raise ValueError("I2_S needs rows divisible by 128")
+    beta = absmean_scale(W)
+    body = interleave_i2s(ternary_codes(W, beta))
+    trailer = np.zeros(TRAILER_BYTES, dtype=np.uint8)
+    trailer[:4] = np.frombuffer(np.asarray([beta], dtype="<f4").tobytes(), dtype=np.uint8)
+    return np.concatenate([body, trailer])
+
+
+def unpack_i2s(packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, np.float32]:
+    """I2_S bytes -> (codes uint8 [N, K], beta)."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    body = packed[: N * K // 4].reshape(N * K // QBLOCK, QBLOCK_BYTES)
+    codes = np.empty((N * K // QBLOCK, 4, QBLOCK_BYTES), dtype=np.uint8)
+    for g in range(4):
+        codes[:, g, :] = (body >> (6 - 2 * g)) & 0x3
+    beta = np.frombuffer(packed[N * K // 4: N * K // 4 + 4].tobytes(), dtype="<f4")[0]
+    return codes.reshape(N, K), F32(beta)
+
+
+# ----------------------------------------------------------------------------- a2: norm + quant
+
+def rmsnorm_quant_act(x: np.ndarray, gain: np.ndarray | None, eps: float):
+    """x fp32 [T, K] (bf16 values widened, or fp32 h) -> (q int8 [T,K], s_x fp32 [T], sum_q int32 [T]).
+
+    With a gain: ms = mean(x^2) (fixed point), inv = 1 / sqrt(ms + eps), y = (x * inv) * g.
+    Without one (use_rms_norm off): y = x.  Then s_x = 127 / max(max|y|, 1e-5),
+    q = clamp(round(y * s_x), -128, 127) and sum_q = sum(q).
+    """
+    x = np.atleast_2d(np.asarray(x, dtype=F32))
+    T, K = x.shape
+    q = np.zeros((T, K), dtype=np.int8)
+    s_x = np.zeros(T, dtype=F32)
+    for t in range(T):
+        row = x[t]
+        if gain is not None:
+            ms = fixed_point_mean_f32(row.astype(F64) * row.astype(F64))
+            inv = F32(1.0) / np.sqrt(ms + F32(eps))
+            y = (row * inv) * np.asarray(gain, dtype=F32)
+        else:
+            y = row
+        a = np.max(np.abs(y)) if K else F32(0.0)
+        s = F32(127.0) / np.maximum(F32(a), ABS_FLOOR)
+        q[t] = np.clip(np.rint(y * s), -128, 127).astype(np.int8)
+        s_x[t] = s
+    sum_q = q.astype(np.int64).sum(axis=1).astype(np.int32)
+    return q, s_x, sum_q
+
+
+# ----------------------------------------------------------------------------- a3/a4: dot + dequant
+
+def bitlinear_acc(q: np.ndarray, sum_q: np.ndarray, packed: np.ndarray, N: int, K: int) -> np.ndarray:
+    """acc[t, n] = sum_k q[t,k] c[n,k] - sum_q[t]  (= sum_k q[t,k] w[n,k], w = c - 1), int32."""
+    codes, _ = unpack_i2s(packed, N, K)
+    qf = np.asarray(q, dtype=F64)
+    acc_c = qf @ codes.astype(F64).T
+    acc = acc_c - np.asarray(sum_q, dtype=F64)[:, None]
+    acc_w = qf @ (codes.astype(F64) - 1.0).T
+    assert np.array_equal(acc, acc_w), "sum q*c - sum q must equal sum q*w"
+    assert np.all(np.abs(acc) < 2 ** 31)
+    return acc.astype(np.int32)
+
+
+def dequant(acc: np.ndarray, s_x: np.ndarray, beta: np.float32) -> np.ndarray:
+    """out = fp32(acc) * (beta / s_x), both fp32 operations."""
+    f = F32(beta) / np.asarray(s_x, dtype=F32)
+    return np.asarray(acc, dtype=np.int32).astype(F32) * f[:, None]
+
+
+def bitlinear(q, s_x, sum_q, packed, N, K, out_dtype="f32", return_acc=False):
+    """One BitLinear after activation quantisation; out fp32 [T, N] (bf16-rounded if asked)."""
+    acc = bitlinear_acc(q, sum_q, packed, N, K)
+    _, beta = unpack_i2s(packed, N, K)
+    out = dequant(acc, s_x, beta)
+    if out_dtype == "bf16":
+        out = round_to_bf16(out)
+    return (out, acc) if return_acc else out
+
+
+# ----------------------------------------------------------------------------- a5: activation
+
+_LN2_DEC = decimal.Context(prec=60).ln(decimal.Decimal(2))  # ln 2 to 60 digits
+_LN2 = float(_LN2_DEC)
+# ln 2 split so that k * _LN2_HI is exact for |k| < 2**11 (Cody and Waite's reduction):
+# _LN2_HI keeps the top 32 significant bits of ln 2, _LN2_LO is the rest, rounded to fp64.
+_LN2_HI = float(np.frombuffer((np.frombuffer(np.float64(_LN2).tobytes(), np.uint64)
+                               & np.uint64(0xFFFFFFFFFFE00000)).tobytes(), np.float64)[0])
+_LN2_LO = float(decimal.Context(prec=60).subtract(_LN2_DEC, decimal.Decimal(_LN2_HI)))
+_EXP_TAYLOR = [1.0 / math.factorial(n) for n in range(18)]  # degree-17 Taylor series of exp
+
+
+def pinned_exp(x: np.ndarray) -> np.ndarray:
+    """exp in fp64 with a fixed operation sequence (so that any IEEE fp64 machine agrees):
+    k = rint(x / ln2); r = (x - k ln2_hi) - k ln2_lo; p = Taylor(r) in Horner form;
+    exp = p * 2**k.  Below -700 the result is 0, above 709 it is +inf."""
+    x = np.asarray(x, dtype=F64)
+    k = np.rint(x / _LN2)
+    r = (x - k * _LN2_HI) - k * _LN2_LO
+    p = np.full_like(r, _EXP_TAYLOR[17])
+    for n in range(16, -1, -1):
+        p = p * r + _EXP_TAYLOR[n]
+    small = x < -700.0
+    big = x > 709.0
+    kk = np.where(small | big, 0, k).astype(np.int64)
+    out = np.ldexp(p, kk)
+    out = np.where(small, 0.0, out)
+    return np.where(big, np.inf, out)
+
+
+def ffn_act(g: np.ndarray, u: np.ndarray, act: str) -> np.ndarray:
+    """h = act(g) * u in fp32.  relu2: r = max(g, 0), h = (r*r)*u.
+    SiLU: s = fp32(g / (1 + exp(-g))) in fp64 with ``pinned_exp``, h = s*u."""
+    g = np.asarray(g, dtype=F32)
+    u = np.asarray(u, dtype=F32)
+    if act == "relu2":
+        r = np.maximum(g, F32(0.0))
+        return (r * r) * u
+    if act == "silu":
+        gd = g.astype(F64)
+        s = (gd / (1.0 + pinned_exp(-gd))).astype(F32)
+        return s * u
+    raise ValueError(act)
+
+
+# ----------------------------------------------------------------------------- composed paths
+
+def bitlinear_from_x(x, gain, eps, packed, N, K, out_dtype="f32"):
+    q, s, sq = rmsnorm_quant_act(x, gain, eps)
+    return bitlinear(q, s, sq, packed, N, K, out_dtype)
+
+
+def ffn_block(x, g_ffn, p_gate, p_up, g_sub, p_down, H, I, act, eps, out_dtype="bf16",
+              return_intermediates=False):
+    """BitNetMLP: down(ffn_sub_norm(act(gate(x)) * up(x))), each projection a BitLinear;
+    gate and up share the quantised input (ffn_norm)."""
+    q, s, sq = rmsnorm_quant_act(x, g_ffn, eps)
+    g = bitlinear(q, s, sq, p_gate, I, H, "f32")
+    u = bitlinear(q, s, sq, p_up, I, H, "f32")
+    h = ffn_act(g, u, act)
+    q2, s2, sq2 = rmsnorm_quant_act(h, g_sub, eps)
+    out = bitlinear(q2, s2, sq2, p_down, H, I, out_dtype)
+    if return_intermediates:
+        return out, dict(q=q, s_x=s, sum_q=sq, g=g, u=u, h=h, q_h=q2, s_h=s2, sum_h=sq2)
+    return out
+
+
+def decoder_block(x, attn_out, gains: dict, packed: dict, shape: dict, act, eps, out_dtype="bf16"):
+    """The BitLinear projections of one decoder block: q,k,v from x through attn_norm;
+    o from the (synthetic) attention output through attn_sub_norm; the FFN from o's
+    output.  ``shape`` maps tensor name -> (N, K).  Returns a dict of outputs."""
+    out = {}
+    q, s, sq = rmsnorm_quant_act(x, gains["attn_norm"], eps)
+    for nm in ("q", "k", "v"):
+        N, K = shape[nm]
+        out[nm] = bitlinear(q, s, sq, packed[nm], N, K, out_dtype)
+    N, K = shape["o"]
+    out["o"] = bitlinear_from_x(attn_out, gains["attn_sub_norm"], eps, packed["o"], N, K, out_dtype)
+    I, H = shape["gate"]
+    out["ffn"] = ffn_block(out["o"], gains["ffn_norm"], packed["gate"], packed["up"],
+                           gains["ffn_sub_norm"], packed["down"], H, I, act, eps, out_dtype)
+    return out

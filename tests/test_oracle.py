@@ -1,0 +1,414 @@
+"""Pins of the CPU oracle to things other than itself (no GPU).
+
+Each test checks the oracle against what the BitNet pages and the mathematics fix:
+hand-worked golden bytes (tests/golden/), exact rational arithmetic, closed forms,
+invariants, special cases that reduce to a library routine, and brute force on tiny
+inputs written independently of the oracle's vectorised code.  The last group plants
+plausible mistakes in the oracle and checks that a pin catches each one.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bitnet_oracle as O
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+F32 = np.float32
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def fraction_to_f32(fr: Fraction) -> np.float32:
+    """Correctly rounded (nearest, ties to even) fp32 of an exact rational."""
+    c = F32(float(fr))
+    best = None
+    for cand in (np.nextafter(c, F32(-np.inf)), c, np.nextafter(c, F32(np.inf))):
+        d = abs(Fraction(float(cand)) - fr)
+        key = (d, int(np.asarray(cand).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, cand)
+    return F32(best[1])
+
+
+def ulp_f32(x) -> float:
+    x = F32(abs(x))
+    return float(np.nextafter(x, F32(np.inf)) - x)
+
+
+def brute_unpack(packed: np.ndarray, N: int, K: int):
+    """Pure-Python decode of the interleaved 128/32 layout, element by element."""
+    data = bytes(np.asarray(packed, dtype=np.uint8)[: N * K // 4])
+    codes = [[None] * K for _ in range(N)]
+    for b in range(N * K // 128):
+        for i in range(32):
+            byte = data[32 * b + i]
+            for g in range(4):
+                flat = 128 * b + 32 * g + i
+                codes[flat // K][flat % K] = (byte >> (6 - 2 * g)) & 3
+    beta = np.frombuffer(bytes(packed[N * K // 4: N * K // 4 + 4]), dtype="<f4")[0]
+    return codes, F32(beta)
+
+
+def read_golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            out[key] = vals
+    return out
+
+
+def bf16_inputs(T, K, seed=0, outliers=False):
+    x = workloads.activations(T, K, seed, "oracle-test", outliers)
+    return O.bf16_bits_to_f32(x.view(torch.int16).numpy().view(np.uint16))
+
+
+# ----------------------------------------------------------------------------- a1: pack
+
+def handworked_weights():
+    k = np.arange(128)
+    w = np.where(k % 3 == 0, F32(0.02), np.where(k % 3 == 1, F32(-0.02), F32(0.0)))
+    return w.astype(F32).reshape(1, 128)
+
+
+def test_pack_handworked_block_golden():
+    g = read_golden("i2s_block_k128.txt")
+    W = handworked_weights()
+    packed = O.pack_i2s(W)
+    assert packed.size == 32 + 32
+    assert [f"{b:02x}" for b in packed[:32]] == g["bytes"]
+    beta_exact = fraction_to_f32(Fraction(int(g["nonzeros"][0])) * Fraction(float(F32(0.02))) / 128)
+    beta = np.frombuffer(packed[32:36].tobytes(), dtype="<f4")[0]
+    assert beta == beta_exact
+    assert not packed[36:].any() and packed[36:].size == int(g["trailer_zero_bytes"][0])
+
+
+def test_pack_zero_tensor_golden():
+    g = read_golden("i2s_zero_tensor.txt")
+    packed = O.pack_i2s(np.zeros((2, 256), F32))
+    assert np.all(packed[: int(g["count"][0])] == int(g["byte"][0], 16))
+    assert np.frombuffer(packed[128:132].tobytes(), "<f4")[0] == F32(float(g["beta_f32"][0]))
+    assert not packed[132:].any()
+
+
+def test_pack_rejects_ragged_rows():
+    with pytest.raises(ValueError):
+        O.pack_i2s(np.zeros((4, 200), F32))
+
+
+def test_packed_size_and_3b_tensor_sizes():
+    g = read_golden("tensor_sizes_3b.txt")
+    for name, (r, c, size, unit) in g.items():
+        nbytes = int(r) * int(c) * 4
+        printed = float(size)
+        got = nbytes / 2 ** 20
+        assert abs(got - printed) <= 0.006 * max(printed, 1), (name, got, printed)
+        if int(c) % 128 == 0 and int(c) > 1:
+            assert O.i2s_packed_bytes(int(r), int(c)) == int(r) * int(c) // 4 + 32
+    # I2_S is 2 bits per weight: 16x below fp32 and 8x below bf16, up to the trailer.
+    assert O.i2s_packed_bytes(3200, 8640) == 6_912_032
+    assert abs(2 * 3200 * 8640 / O.i2s_packed_bytes(3200, 8640) - 8.0) < 1e-4
+
+
+@pytest.mark.parametrize("N,K,seed", [(3, 128, 0), (5, 256, 1), (17, 384, 2), (64, 1024, 3)])
+def test_pack_matches_bruteforce_decode(N, K, seed):
+    W = workloads.latent_weight(N, K, seed, "pin").numpy()
+    packed = O.pack_i2s(W)
+    assert packed.size == N * K // 4 + 32
+    codes, beta = brute_unpack(packed, N, K)
+    # Independent codes: round-half-even of W / beta in exact arithmetic for the same fp32 s_w.
+    s_w = F32(1.0) / beta
+    for n in range(N):
+        for k in range(K):
+            prod = Fraction(float(W[n, k])) * Fraction(float(s_w))
+            v = float(F32(float(prod)))  # fp32 product, correctly rounded
+            want = max(-1, min(1, round(fraction_to_f32(Fraction(v)).item()))) + 1
+            assert codes[n][k] == want, (n, k)
+    vc, vb = O.unpack_i2s(packed, N, K)
+    assert vb == beta and np.array_equal(vc, np.array(codes, dtype=np.uint8))
+
+
+@pytest.mark.parametrize("N,K,seed", [(8, 256, 0), (33, 512, 1), (100, 1280, 2)])
+def test_beta_is_exact_mean_rounded(N, K, seed):
+    W = workloads.latent_weight(N, K, seed, "beta").numpy()
+    exact = sum(Fraction(float(abs(v))) for v in W.ravel()) / (N * K)
+    beta = O.absmean_scale(W)
+    want = fraction_to_f32(exact)
+    assert abs(float(beta) - float(want)) <= ulp_f32(want), (beta, want)
+
+
+@pytest.mark.parametrize("alpha", [1e-4, 3e-3, 0.0123, 0.5, 1.0, 7.25, 300.0])
+def test_scale_invariance_of_ternary_inputs(alpha):
+    rng = np.random.default_rng(int(alpha * 1e4) % 2**31)
+    T = rng.integers(-1, 2, size=(6, 256)).astype(F32)
+    T[0, :] = 0.0
+    T[0, 5] = 1.0  # a row with a single non-zero
+    packed = O.pack_i2s(F32(alpha) * T)
+    codes, beta = brute_unpack(packed, 6, 256)
+    assert np.array_equal(np.array(codes) - 1, T.astype(int))
+    # Re-packing the dequantised tensor keeps the codes (ternary x scale is a fixed point).
+    W2 = (np.array(codes, dtype=F32) - 1) * beta
+    assert np.array_equal(O.pack_i2s(W2)[: 6 * 256 // 4], packed[: 6 * 256 // 4])
+
+
+# ----------------------------------------------------------------------------- a2: norm + quant
+
+@pytest.mark.parametrize("K,seed", [(128, 0), (2560, 1), (6912, 2)])
+def test_mean_square_is_exact_mean_rounded(K, seed):
+    x = bf16_inputs(3, K, seed)
+    for t in range(3):
+        exact = sum(Fraction(float(v)) ** 2 for v in x[t]) / K
+        ms = O.fixed_point_mean_f32(x[t].astype(np.float64) ** 2)
+        want = fraction_to_f32(exact)
+        assert abs(float(ms) - float(want)) <= ulp_f32(want)
+
+
+def test_fixed_point_sum_is_order_free_and_bounded():
+    rng = np.random.default_rng(0)
+    v = np.abs(rng.standard_normal(10_000)) ** 3
+    S1, e1 = O.fixed_point_sum(v)
+    S2, e2 = O.fixed_point_sum(v[::-1].copy())
+    S3, e3 = O.fixed_point_sum(rng.permutation(v))
+    assert S1 == S2 == S3 and e1 == e2 == e3
+    assert 0 < S1 < 2 ** 62
+    assert abs(math.ldexp(S1, -e1) - math.fsum(v)) <= 10_000 * math.ldexp(1.0, -e1)
+
+
+@pytest.mark.parametrize("use_norm", [True, False])
+def test_quant_invariants(use_norm):
+    T, K = 7, 640
+    x = bf16_inputs(T, K, 4)
+    x[3] = 0.0  # a zero token
+    g = workloads.gain(K, 0, "pin").numpy() if use_norm else None
+    q, s, sq = O.rmsnorm_quant_act(x, g, 1e-6)
+    assert q.dtype == np.int8 and s.dtype == F32 and sq.dtype == np.int32
+    for t in range(T):
+        if t == 3:
+            assert not q[t].any() and s[t] == F32(127.0) / F32(1e-5) and sq[t] == 0
+            continue
+        xd = x[t].astype(np.float64)
+        y = xd / math.sqrt(np.mean(xd * xd) + 1e-6) * g.astype(np.float64) if use_norm else xd
+        a = np.max(np.abs(y))
+        assert abs(float(s[t]) - 127.0 / a) <= 1e-6 * 127.0 / a
+        assert np.max(np.abs(q[t])) == 127
+        assert np.abs(q[t][np.argmax(np.abs(y))]) == 127
+        assert np.all(np.abs(q[t] - y * 127.0 / a) <= 0.5 + 1e-4)
+        assert sq[t] == int(q[t].astype(np.int64).sum())
+
+
+def test_quant_without_gain_is_plain_absmax():
+    x = bf16_inputs(2, 256, 9)
+    q, s, _ = O.rmsnorm_quant_act(x, None, 1e-6)
+    for t in range(2):
+        a = max(abs(float(v)) for v in x[t])
+        assert s[t] == fraction_to_f32(Fraction(127) / Fraction(float(F32(a))))
+        for k in range(256):
+            exact = Fraction(float(x[t, k])) * Fraction(float(s[t]))
+            v = float(F32(float(exact)))  # the fp32 product, correctly rounded
+            assert q[t, k] == max(-128, min(127, round(v)))
+
+
+def test_quant_ties_round_half_even():
+    # amax = 127/64 makes s_x = 64 exactly, so x = (n + 0.5)/64 lands on a tie.
+    x = np.zeros((1, 128), F32)
+    x[0, 0] = F32(127.0 / 64.0)
+    halves = [0.5, 1.5, 2.5, 3.5, -0.5, -1.5, -2.5, 100.5]
+    for i, h in enumerate(halves):
+        x[0, 1 + i] = F32(h / 64.0)
+    q, s, _ = O.rmsnorm_quant_act(x, None, 1e-6)
+    assert s[0] == F32(64.0)
+    assert list(q[0, 1:1 + len(halves)]) == [0, 2, 2, 4, 0, -2, -2, 100]
+
+
+def test_rmsnorm_matches_textbook():
+    x = bf16_inputs(4, 2560, 5)
+    g = workloads.gain(2560, 0, "pin").numpy()
+    # y is not returned; check through s_x, which is 127 / max|y|.
+    _, s, _ = O.rmsnorm_quant_act(x, g, 1e-6)
+    for t in range(4):
+        xd = x[t].astype(np.float64)
+        y = xd / math.sqrt(float(np.mean(xd * xd)) + 1e-6) * g.astype(np.float64)
+        assert abs(float(s[t]) * np.max(np.abs(y)) - 127.0) <= 127.0 * 4e-7
+
+
+# ----------------------------------------------------------------------------- a3/a4: dot + dequant
+
+@pytest.mark.parametrize("T,N,K,seed", [(1, 1, 128, 0), (2, 3, 128, 1), (3, 4, 256, 2), (4, 2, 384, 3)])
+def test_dot_bruteforce(T, N, K, seed):
+    W = workloads.latent_weight(N, K, seed, "dot").numpy()
+    packed = O.pack_i2s(W)
+    x = bf16_inputs(T, K, seed)
+    q, s, sq = O.rmsnorm_quant_act(x, None, 1e-6)
+    acc = O.bitlinear_acc(q, sq, packed, N, K)
+    codes, beta = brute_unpack(packed, N, K)
+    out = O.bitlinear(q, s, sq, packed, N, K, "f32")
+    for t in range(T):
+        for n in range(N):
+            want = sum(int(q[t, k]) * (codes[n][k] - 1) for k in range(K))
+            assert acc[t, n] == want
+            # Dequantised value in exact arithmetic: acc * beta / s_x.
+            exact = Fraction(want) * Fraction(float(beta)) / Fraction(float(s[t]))
+            if want == 0:
+                assert out[t, n] == 0
+            else:
+                assert abs(Fraction(float(out[t, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 22)
+
+
+@pytest.mark.parametrize("T", [1, 3, 16])
+def test_bitlinear_matches_textbook_gemv(T):
+    N, K = 96, 1024
+    W = workloads.latent_weight(N, K, T, "gemv").numpy()
+    packed = O.pack_i2s(W)
+    x = bf16_inputs(T, K, T)
+    g = workloads.gain(K, T, "gemv").numpy()
+    q, s, sq = O.rmsnorm_quant_act(x, g, 1e-6)
+    codes, beta = O.unpack_i2s(packed, N, K)
+    # Textbook: dequantise both operands in fp64 and take the plain matrix product.
+    xq = q.astype(np.float64) / s.astype(np.float64)[:, None]
+    wq = (codes.astype(np.float64) - 1.0) * float(beta)
+    ref = xq @ wq.T
+    # fp64 rounding of the textbook sum: a few ulp of the sum of |terms|.
+    slack = 1e-14 * (np.abs(xq) @ np.abs(wq).T)
+    for dt, tol in (("f32", 1e-6), ("bf16", 2.0 ** -8)):
+        out = O.bitlinear(q, s, sq, packed, N, K, dt).astype(np.float64)
+        assert np.all(np.abs(out - ref) <= tol * np.abs(ref) + slack)
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.standard_normal(100_000).astype(F32) * 10.0 ** rng.integers(-30, 30, 100_000),
+                        np.array([0.0, -0.0, 1.0, 1.00390625, 1.005859375, 3.0e38], F32)]).astype(F32)
+    got = O.f32_to_bf16_bits(v)
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.bf16_bits_to_f32(got), torch.from_numpy(v).to(torch.bfloat16).float().numpy())
+
+
+# ----------------------------------------------------------------------------- a5: activation
+
+def test_pinned_exp_against_libm():
+    xs = np.concatenate([np.linspace(-700, 709, 200_001), np.array([0.0, 1.0, -1.0, math.log(2.0), 1e-300])])
+    got = O.pinned_exp(xs)
+    want = np.array([math.exp(v) for v in xs])
+    rel = np.abs(got - want) / want
+    assert np.max(rel) <= 4e-15
+    assert O.pinned_exp(np.array([0.0]))[0] == 1.0
+    assert O.pinned_exp(np.array([-800.0]))[0] == 0.0 and np.isinf(O.pinned_exp(np.array([710.0]))[0])
+
+
+def test_silu_matches_torch():
+    g = (np.random.default_rng(1).standard_normal(50_000) * 8).astype(F32)
+    h = O.ffn_act(g, np.ones_like(g), "silu")
+    ref = torch.nn.functional.silu(torch.from_numpy(g).double()).numpy()
+    err = np.abs(h.astype(np.float64) - ref)
+    assert np.all(err <= np.array([ulp_f32(v) for v in ref]) * 0.5 + 1e-45)
+
+
+def test_relu2_closed_form():
+    rng = np.random.default_rng(2)
+    g = rng.standard_normal(20_000).astype(F32)
+    u = rng.standard_normal(20_000).astype(F32)
+    h = O.ffn_act(g, u, "relu2").astype(np.float64)
+    ref = np.where(g > 0, g.astype(np.float64) ** 2 * u, 0.0)
+    assert np.all(h[g <= 0] == 0)
+    assert np.max(np.abs(h - ref) / np.maximum(np.abs(ref), 1e-30)) <= 2.5e-7
+
+
+# ----------------------------------------------------------------------------- composed: FFN
+
+def textbook_ffn(x, g_ffn, W_gate, W_up, g_sub, W_down, act, eps=1e-6):
+    """BitNetMLP in fp64 from the plain formulas: RMSNorm, absmax int8, absmean ternary."""
+    def norm_quant(v, gain):
+        v = v.astype(np.float64)
+        y = v / np.sqrt(np.mean(v * v, axis=1, keepdims=True) + eps) * gain.astype(np.float64)
+        s = 127.0 / np.maximum(np.max(np.abs(y), axis=1, keepdims=True), 1e-5)
+        return np.clip(np.round(y * s), -128, 127) / s
+
+    def ternary(W):
+        W = W.astype(np.float64)
+        beta = max(np.mean(np.abs(W)), 1e-5)
+        return np.clip(np.round(W / beta), -1, 1) * beta
+
+    xq = norm_quant(x, g_ffn)
+    gt, up = xq @ ternary(W_gate).T, xq @ ternary(W_up).T
+    a = np.maximum(gt, 0.0) ** 2 if act == "relu2" else gt / (1.0 + np.exp(-gt))
+    hq = norm_quant(a * up, g_sub)
+    return hq @ ternary(W_down).T
+
+
+@pytest.mark.parametrize("act", ["relu2", "silu"])
+def test_ffn_block_matches_textbook(act):
+    H, I, T = 256, 640, 3
+    d = {nm: workloads.latent_weight(n, k, 7, "ffn/" + nm).numpy()
+         for nm, (n, k) in {"gate": (I, H), "up": (I, H), "down": (H, I)}.items()}
+    x = bf16_inputs(T, H, 7)
+    g1 = workloads.gain(H, 7, "ffn1").numpy()
+    g2 = workloads.gain(I, 7, "ffn2").numpy()
+    p = {nm: O.pack_i2s(W) for nm, W in d.items()}
+    out = O.ffn_block(x, g1, p["gate"], p["up"], g2, p["down"], H, I, act, 1e-6, "f32")
+    ref = textbook_ffn(x, g1, d["gate"], d["up"], g2, d["down"], act)
+    assert np.linalg.norm(out - ref) / np.linalg.norm(ref) <= 2e-3
+
+
+def test_decoder_block_runs_and_chains():
+    sh = workloads.BlockShape("tiny", hidden=256, n_q=256, n_kv=128, inter=384, act="relu2")
+    d = workloads.block_inputs(sh, T=2, seed=3)
+    packed = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in sh.tensors()}
+    gains = {k[2:]: v.numpy() for k, v in d.items() if k.startswith("g_")}
+    xb = O.bf16_bits_to_f32(d["x"].view(torch.int16).numpy().view(np.uint16))
+    ab = O.bf16_bits_to_f32(d["attn_out"].view(torch.int16).numpy().view(np.uint16))
+    out = O.decoder_block(xb, ab, gains, packed, sh.tensors(), "relu2", 1e-6, "bf16")
+    assert out["q"].shape == (2, 256) and out["k"].shape == (2, 128) and out["ffn"].shape == (2, 256)
+    ffn = O.ffn_block(out["o"], gains["ffn_norm"], packed["gate"], packed["up"], gains["ffn_sub_norm"],
+                      packed["down"], 256, 384, "relu2", 1e-6, "bf16")
+    assert np.array_equal(ffn, out["ffn"])
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+
+def _sequential_interleave(codes):
+    N, K = codes.shape
+    c = codes.reshape(-1, 4).astype(np.uint8)  # byte i/4, field i%4
+    return ((c[:, 0] << 6) | (c[:, 1] << 4) | (c[:, 2] << 2) | c[:, 3]).astype(np.uint8)
+
+
+@pytest.mark.parametrize("mutant", ["sequential_layout", "codes_minus_one", "no_half_even",
+                                    "mean_without_divide", "transposed_dot", "gate_up_swapped"])
+def test_pins_catch_planted_mistakes(monkeypatch, mutant):
+    if mutant == "sequential_layout":
+        monkeypatch.setattr(O, "interleave_i2s", _sequential_interleave)
+        check = test_pack_handworked_block_golden
+    elif mutant == "codes_minus_one":
+        orig = O.ternary_codes
+        monkeypatch.setattr(O, "ternary_codes", lambda W, b: (orig(W, b).astype(np.int16) - 1).astype(np.uint8) & 3)
+        check = test_pack_handworked_block_golden
+    elif mutant == "no_half_even":
+        monkeypatch.setattr(O.np, "rint", lambda v: np.floor(np.asarray(v) + 0.5))
+        check = test_quant_ties_round_half_even
+    elif mutant == "mean_without_divide":
+        monkeypatch.setattr(O, "fixed_point_mean_f32",
+                            lambda t: F32(math.ldexp(float(O.fixed_point_sum(t)[0]), -O.fixed_point_sum(t)[1])))
+        check = lambda: test_mean_square_is_exact_mean_rounded(128, 0)
+    elif mutant == "transposed_dot":
+        orig_unpack = O.unpack_i2s
+        def bad(packed, N, K):
+            c, b = orig_unpack(packed, N, K)
+            return c[:, ::-1].copy(), b
+        monkeypatch.setattr(O, "unpack_i2s", bad)
+        check = lambda: test_dot_bruteforce(2, 3, 128, 1)
+    else:
+        orig_ffn_act = O.ffn_act
+        monkeypatch.setattr(O, "ffn_act", lambda g, u, act: orig_ffn_act(u, g, act))
+        check = lambda: test_ffn_block_matches_textbook("relu2")
+    with pytest.raises(AssertionError):
+        check()
