@@ -1,0 +1,476 @@
+"""Benchmark of the BitNet b1.58 BitLinear forward on B200.
+
+Default workload: the 2B4T-shaped decoder block at decode (T = 1): q,k,v (attn_norm,
+one grouped launch), o (attn_sub_norm, on a synthetic attention output), and the FFN
+(ffn_norm -> gate/up -> relu2 -> ffn_sub_norm -> down, fed by o's output).  A step is
+one pass of that whole path; weights are packed once before timing (offline step).
+
+value  = packed-weight bytes read per step x steps x ranks / device time (max over ranks)
+         [GB/s]; for prefill workloads (T >= 64) int8 TOPS = 2 T sum(N K) / time.
+e2e    = the same metric with each step's activations copied from pinned host memory
+         and its outputs copied back, inside the timed region.
+L2     = the packed weights rotate over enough copies to exceed 2x the 126 MB L2, so
+         every step reads its weights from HBM.
+
+``--impl reference`` times the CPU oracle (numpy) on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="block_2b4t_decode_t1", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle sample")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [ln.split(",") for ln in self.f.read().strip().splitlines() if ln.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel_key: str, sha: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)
+        e = d.get(kernel_key)
+        if e and e.get("source_sha") == sha:
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------------------- workload on the GPU
+
+class Workload:
+    def __init__(self, name: str, seed: int, device: str):
+        import ternary_bitlinear_quantized_b200 as tb
+        self.tb = tb
+        self.name = name
+        self.spec = workloads.WORKLOADS[name]
+        self.kind = self.spec["kind"]
+        self.T = self.spec["T"]
+        dev = device
+        self.dev = dev
+        if self.kind == "bitlinear":
+            N, K = self.spec["N"], self.spec["K"]
+            self.tensors = {"w": (N, K)}
+            W = {"w": workloads.latent_weight(N, K, seed, name, dev)}
+            self.x = workloads.activations(self.T, K, seed, name + "/x", device=dev)
+            self.g = workloads.gain(K, seed, name + "/g", dev)
+        else:
+            sh = self.spec["shape"]
+            self.shape = sh
+            ffn_only = self.kind == "ffn"
+            d = workloads.block_inputs(sh, self.T, seed, self.spec.get("outliers", False), dev, ffn_only)
+            self.d = d
+            self.tensors = {nm: sh.tensors()[nm] for nm in (["gate", "up", "down"] if ffn_only else sh.tensors())}
+            W = {nm: d["W_" + nm] for nm in self.tensors}
+            self.act = tb.RELU2 if sh.act == "relu2" else tb.SILU
+        self.packed_bytes = sum(tb.i2s_packed_bytes(n, k) for (n, k) in self.tensors.values())
+        self.ops_per_step = sum(2 * self.T * n * k for (n, k) in self.tensors.values())
+        # Pack once (offline), then replicate the bytes so that the copies exceed 2x L2.
+        packed = {nm: tb.pack_i2s(W[nm]) for nm in self.tensors}
+        del W
+        self.n_copies = max(1, math.ceil(2 * L2_BYTES / self.packed_bytes) + 1)
+        self.copies = [packed] + [{nm: p.clone() for nm, p in packed.items()} for _ in range(self.n_copies - 1)]
+        self._alloc_outputs()
+
+    def _alloc_outputs(self):
+        T, dev = self.T, self.dev
+        e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=dev)
+        if self.kind == "bitlinear":
+            N, K = self.tensors["w"]
+            self.qbuf = (e(T, K, dt=torch.int8), e(T, dt=torch.float32), e(T, dt=torch.int32))
+            self.out = e(T, N)
+            self.outputs = [self.out]
+            self.inputs = [self.x]
+            return
+        sh = self.shape
+        H, I = sh.hidden, sh.inter
+        if self.kind == "block":
+            self.qx = (e(T, H, dt=torch.int8), e(T, dt=torch.float32), e(T, dt=torch.int32))
+            self.qa = (e(T, sh.n_q, dt=torch.int8), e(T, dt=torch.float32), e(T, dt=torch.int32))
+            self.oq, self.ok_, self.ov = e(T, sh.n_q), e(T, sh.n_kv), e(T, sh.n_kv)
+            self.oo = e(T, H)
+            self.inputs = [self.d["x"], self.d["attn_out"]]
+        else:
+            self.inputs = [self.d["x"]]
+        self.offn = e(T, H)
+        self.ws = torch.empty(self.tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=self.dev)
+        self.outputs = ([self.oq, self.ok_, self.ov, self.offn] if self.kind == "block" else [self.offn])
+
+    def step(self, c: int):
+        tb, p = self.tb, self.copies[c]
+        if self.kind == "bitlinear":
+            q, s, sq = tb.rmsnorm_quant_act(self.x, self.g, workloads.EPS, out=self.qbuf)
+            tb.bitlinear(q, s, sq, p["w"], self.tensors["w"][0], out=self.out)
+            return
+        d, sh = self.d, self.shape
+        ffn_in = d["x"]
+        if self.kind == "block":
+            q, s, sq = tb.rmsnorm_quant_act(d["x"], d["g_attn_norm"], workloads.EPS, out=self.qx)
+            tb.bitlinear_group(q, s, sq, [p["q"], p["k"], p["v"]], [sh.n_q, sh.n_kv, sh.n_kv],
+                               outs=[self.oq, self.ok_, self.ov])
+            q, s, sq = tb.rmsnorm_quant_act(d["attn_out"], d["g_attn_sub_norm"], workloads.EPS, out=self.qa)
+            tb.bitlinear(q, s, sq, p["o"], sh.hidden, out=self.oo)
+            ffn_in = self.oo
+        tb.ffn_block(ffn_in, d["g_ffn_norm"], p["gate"], p["up"], d["g_ffn_sub_norm"], p["down"], sh.inter,
+                     self.act, workloads.EPS, out=self.offn, ws=self.ws)
+
+    def launches_per_step(self) -> int:
+        return {"bitlinear": 2, "block": 8, "ffn": 4}[self.kind]
+
+    def dominant(self):
+        """(label, callable(c), bytes per launch, ops per launch) of the largest product kernel:
+        the FFN's gate/up launch (relu2/SiLU epilogue) or the single BitLinear."""
+        tb = self.tb
+        if self.kind == "bitlinear":
+            N, K = self.tensors["w"]
+            q, s, sq = self.qbuf
+            return ("k_gemv_mma (bitlinear)", lambda c: tb.bitlinear(q, s, sq, self.copies[c]["w"], N, out=self.out),
+                    tb.i2s_packed_bytes(N, K), 2 * self.T * N * K)
+        sh = self.shape
+        H, I = sh.hidden, sh.inter
+        off = tb.ffn_workspace_offsets(self.T, H, I)
+        T = self.T
+        q = self.ws[off[0]:off[0] + T * H].view(torch.int8).view(T, H)
+        s = self.ws[off[1]:off[1] + 4 * T].view(torch.float32)
+        sq = self.ws[off[2]:off[2] + 4 * T].view(torch.int32)
+        h = self.ws[off[3]:off[3] + 4 * T * I].view(torch.float32).view(T, I)
+        fn = lambda c: tb.bitlinear_gate_up_act(q, s, sq, self.copies[c]["gate"], self.copies[c]["up"], I, self.act,
+                                                out=h)
+        return ("k_gemv_mma<ffn> (gate/up + act)", fn, 2 * tb.i2s_packed_bytes(I, H), 4 * T * I * H)
+
+
+def time_steps(wl: Workload, steps: int, warmup: int, use_graph: bool, e2e: bool):
+    """Device time (ms) of `steps` steps, after `warmup` untimed ones."""
+    R = wl.n_copies
+    host_in = [t.cpu().pin_memory() for t in wl.inputs] if e2e else None
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in wl.outputs] if e2e else None
+
+    def one(c):
+        if e2e:
+            for h, d in zip(host_in, wl.inputs):
+                d.copy_(h, non_blocking=True)
+        wl.step(c)
+        if e2e:
+            for h, d in zip(host_out, wl.outputs):
+                h.copy_(d, non_blocking=True)
+
+    for c in range(min(R, 2)):
+        one(c)
+    torch.cuda.synchronize()
+    graphs = None
+    if use_graph:
+        graphs = []
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        for c in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                one(c)
+            graphs.append(g)
+        torch.cuda.synchronize()
+    run = (lambda i: graphs[i % R].replay()) if use_graph else (lambda i: one(i % R))
+    for i in range(warmup):
+        run(i)
+    torch.cuda.synchronize()
+    if torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(steps):
+        run(warmup + i)
+    ev1.record()
+    torch.cuda.synchronize()
+    if torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    ms = ev0.elapsed_time(ev1)
+    del graphs
+    h2d = sum(t.numel() * t.element_size() for t in wl.inputs) if e2e else 0
+    d2h = sum(t.numel() * t.element_size() for t in wl.outputs) if e2e else 0
+    return ms, h2d, d2h
+
+
+def time_dominant(wl: Workload, launches: int):
+    """Average device duration of the dominant kernel, launched alone (weights rotating)."""
+    label, fn, nbytes, ops = wl.dominant()
+    R = wl.n_copies
+    for c in range(min(R, 3)):
+        fn(c)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    stream = torch.cuda.current_stream()
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        fn(i % R)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return label, statistics.mean(ms), nbytes, ops
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(name: str, seed: int, seconds: float):
+    """Time the numpy oracle on this workload (bounded sample).  Returns (units/s, unit, sample, cores)."""
+    import numpy as np
+    from oracle import bitnet_oracle as O
+    spec = workloads.WORKLOADS[name]
+    T = spec["T"]
+    decode = T < 64
+    if spec["kind"] == "bitlinear":
+        N, K = spec["N"], spec["K"]
+        W = workloads.latent_weight(N, K, seed, name).numpy()
+        packed = O.pack_i2s(W)
+        x = workloads.activations(T, K, seed, name + "/x")
+        xf = O.bf16_bits_to_f32(x.view(torch.int16).numpy().view(np.uint16))
+        g = workloads.gain(K, seed, name + "/g").numpy()
+        tensors = {"w": (N, K)}
+        run = lambda xs: O.bitlinear_from_x(xs, g, workloads.EPS, packed, N, K, "bf16")
+    else:
+        sh = spec["shape"]
+        ffn_only = spec["kind"] == "ffn"
+        d = workloads.block_inputs(sh, T, seed, spec.get("outliers", False), "cpu", ffn_only)
+        tensors = {nm: sh.tensors()[nm] for nm in (["gate", "up", "down"] if ffn_only else sh.tensors())}
+        packed = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in tensors}
+        gains = {k[2:]: v.numpy() for k, v in d.items() if k.startswith("g_")}
+        xf = O.bf16_bits_to_f32(d["x"].view(torch.int16).numpy().view(np.uint16))
+        af = None if ffn_only else O.bf16_bits_to_f32(d["attn_out"].view(torch.int16).numpy().view(np.uint16))
+        H, I = sh.hidden, sh.inter
+        if ffn_only:
+            run = lambda xs, a=None: O.ffn_block(xs, gains["ffn_norm"], packed["gate"], packed["up"],
+                                                 gains["ffn_sub_norm"], packed["down"], H, I, sh.act,
+                                                 workloads.EPS, "bf16")
+        else:
+            run = lambda xs, a=None: O.decoder_block(xs, a, gains, packed, sh.tensors(), sh.act, workloads.EPS,
+                                                     "bf16")
+    pbytes = sum(n * k // 4 + 32 for (n, k) in tensors.values())
+    # Tokens are independent through every step, so a prefill sample takes a few tokens.
+    t_sample = T if decode else min(T, 8)
+    xs = xf[:t_sample]
+    a_s = None if spec["kind"] != "block" else af[:t_sample]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        if spec["kind"] == "block":
+            run(xs, a_s)
+        else:
+            run(xs)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    if decode:
+        val = pbytes * n / el / 1e9
+        unit = "GB/s"
+        sample = f"{n} full steps of the workload (T={T}) in {el:.1f} s"
+    else:
+        ops = sum(2 * t_sample * nn * kk for (nn, kk) in tensors.values())
+        val = ops * n / el / 1e12
+        unit = "TOPS"
+        sample = f"{n} steps on {t_sample} of the {T} tokens (tokens are independent) in {el:.1f} s"
+    return val, unit, sample, cores
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = workloads.WORKLOADS[args.workload]
+    decode = spec["T"] < 64
+    metric = ("packed-weight HBM GB/s (decode)" if decode else "int8 TOPS (prefill)")
+    unit = "GB/s" if decode else "TOPS"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        val, u, sample, cores = oracle_sample(args.workload, args.seed, args.cpu_seconds)
+        line = {"metric": metric, "value": val, "unit": u, "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "impl": "reference", "dtype": "int8", "data": "synthetic",
+                "config": {"workload": args.workload, "T": spec["T"]},
+                "cpu_baseline": {"value": val, "unit": u, "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": val, "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from ternary_bitlinear_quantized_b200 import build as tbuild
+    if rank == 0 or world == 1:
+        tbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    wl = Workload(args.workload, args.seed + 0, f"cuda:{local}")  # same workload on every rank (replicas)
+    use_graph = not args.no_graph
+
+    clk = ClockSampler(local)
+    clk.start()
+    ms, _, _ = time_steps(wl, args.steps, args.warmup, use_graph, e2e=False)
+    clocks = clk.stop()
+    ms_e2e, h2d, d2h = time_steps(wl, args.steps, args.warmup, use_graph, e2e=True)
+    label, dom_ms, dom_bytes, dom_ops = time_dominant(wl, max(50, min(args.steps, 500)))
+    status = wl.tb.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms, ms_e2e = float(t[0]), float(t[1])
+    per_step_units = wl.packed_bytes / 1e9 if decode else wl.ops_per_step / 1e12
+    value = world * per_step_units * args.steps / (ms / 1e3)
+    e2e_val = world * per_step_units * args.steps / (ms_e2e / 1e3)
+
+    hbm, bf16, src = peaks()
+    kernel_files = ["ternary_bitlinear_quantized_b200/csrc/gemv.cuh", "ternary_bitlinear_quantized_b200/csrc/common.cuh"]
+    if decode:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": stored_traffic(label, source_sha(kernel_files)), "kernel": label,
+                "bytes_per_launch": dom_bytes, "launch_us": dom_ms * 1e3,
+                "peak_source": f"{src} hbm_gbs (copy bandwidth, burst)"}
+    else:
+        achieved = dom_ops / (dom_ms / 1e3) / 1e12
+        int8_peak = bf16 * 2.0  # dense int8 = 2x dense bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak,
+                "traffic": stored_traffic(label, source_sha(kernel_files)), "kernel": label,
+                "ops_per_launch": dom_ops, "launch_us": dom_ms * 1e3,
+                "peak_source": f"{src} bf16_tflops x 2 (nominal int8/bf16 ratio)"}
+
+    cpu = None
+    if rank == 0 and world == 1:
+        val, u, sample, cores = oracle_sample(args.workload, args.seed, args.cpu_seconds)
+        cpu = {"value": val, "unit": u, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": args.workload, "T": wl.T, "packed_bytes_per_step": wl.packed_bytes,
+                       "int8_ops_per_step": wl.ops_per_step, "parallelism": f"replicas x{world}",
+                       "l2": f"weights rotated over {wl.n_copies} copies "
+                             f"({wl.n_copies * wl.packed_bytes / 1e6:.0f} MB > 2x L2)",
+                       "cuda_graphs": use_graph},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": wl.launches_per_step() * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,176 @@
+/*
+ * bitnet_b200.h -- C ABI of the BitNet b1.58 BitLinear forward on NVIDIA B200 (sm_100a).
+ *
+ * The forward of one BitLinear: an RMSNorm on the activations (optional), per-token
+ * absmax int8 quantisation of the activations, the integer product with absmean-ternary
+ * weights stored as 2-bit I2_S codes, and the dequantising rescale.  On top of it, the
+ * BitNet FFN block: gate/up -> relu2 or SiLU -> ffn_sub_norm -> down.
+ *
+ * Sources (web pages, by title):
+ *   [RMS]  "Add optional RMSNorm support to BitNet quantization (config + layers)"
+ *          (transformers pull request 38087): use_rms_norm (default off) and
+ *          rms_norm_eps (default 1e-6); BitLinear applies BitNetRMSNorm to the
+ *          activations before quantisation; BitNetMLP.forward (review thread).
+ *   [I2S]  "fix: I2_S ARM kernel layout + squared-ReLU FFN - passes the gate on the
+ *          official 2B4T GGUF" (cpp-bitnet pull request 7): description bullets
+ *          "I2_S NEON kernel for the canonical layout" (interleaved 128-weight / 32-byte
+ *          blocks, codes c = w + 1, the callers subtract the activation sum),
+ *          "llama-quantize I2_S emits the canonical layout" (one scale per tensor after
+ *          the packed data, 28 zeroed trailer bytes), "squared-ReLU FFN" (relu2 vs
+ *          SiLU chosen from config) and "Known gaps" (rows divisible by 128).
+ *   [IQ1]  "More BitNet-like IQ1_S quantizations" (llama.cpp discussion 8722):
+ *          BitNet b1.58 keeps 8-bit activations and ternary weights.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated otherwise, 16-byte aligned, to
+ *     contiguous row-major tensors.  The caller allocates and owns every buffer; the
+ *     library allocates no device memory.
+ *   - Calls are asynchronous on stream `s` (a cudaStream_t; NULL = legacy default
+ *     stream).  Kernels are launched with programmatic dependent launch: a kernel may
+ *     start, and read its WEIGHTS (`packed`) and norm GAINS, while the previous kernel
+ *     on `s` is still running; it reads activations only after that kernel has
+ *     finished.  So weights and gains must not be written by the kernel that directly
+ *     precedes the call on `s` unless that kernel finishes before this one is enqueued
+ *     (any torch kernel or copy satisfies this; so does bitnet_pack_i2s).
+ *   - Argument errors are returned before anything is launched.  A launch failure
+ *     returns BITNET_ERR_CUDA; bitnet_last_error() gives the CUDA message (per thread).
+ *   - T = 0 (no tokens) is valid and launches nothing.
+ *   - Entry points are reentrant; the only global state is the device status word read
+ *     by bitnet_get_device_status().
+ */
+#ifndef BITNET_B200_H
+#define BITNET_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bitnet_stream; /* the same handle as cudaStream_t */
+
+typedef enum {
+  BITNET_OK = 0,
+  BITNET_ERR_NULL = 1,      /* a required pointer is NULL                               */
+  BITNET_ERR_SHAPE = 2,     /* a size is negative/zero where it must be positive, K % 128 != 0 for
+                               packed weights, or a size is beyond the supported maximum   */
+  BITNET_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned                          */
+  BITNET_ERR_DTYPE = 4,     /* unknown bitnet_dtype / bitnet_act value                    */
+  BITNET_ERR_WORKSPACE = 5, /* workspace missing or smaller than the *_workspace_bytes() */
+  BITNET_ERR_CUDA = 6,      /* a CUDA call failed; see bitnet_last_error()               */
+  BITNET_ERR_TIMEOUT = 7    /* a kernel gave up a bounded wait (device status word)      */
+} bitnet_status;
+
+typedef enum { BITNET_BF16 = 0, BITNET_F32 = 1 } bitnet_dtype;
+typedef enum { BITNET_RELU2 = 0, BITNET_SILU = 1 } bitnet_act;
+
+/* Largest in-feature count K the norm/quant kernels accept (a whole row is staged in
+ * shared memory as fp32). */
+#define BITNET_MAX_K 49152
+
+/* Size of an I2_S tensor of N rows and K in-features: N*K/4 bytes of codes followed by
+ * a 32-byte trailer (fp32 scale, then 28 zero bytes).  [I2S] "llama-quantize I2_S emits
+ * the canonical layout".  Returns 0 if N <= 0, K <= 0 or K % 128 != 0. */
+size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K);
+
+/* Ternarise and pack latent fp32 weights W [N, K] into I2_S (`packed`, which must hold
+ * bitnet_i2s_packed_bytes(N, K) bytes).
+ *   beta = max(mean|W|, 1e-5)   (the mean is an exact fixed-point sum rounded once to fp32)
+ *   s_w  = 1 / beta;  c = clamp(round_half_even(W * s_w), -1, 1) + 1  in {0, 1, 2}
+ *   element k of row n (block b = (n*K + k) / 128, g = (k % 128) / 32, i = k % 32) goes to
+ *   byte 32 b + i, bits (7 - 2g):(6 - 2g); fp32 beta (little endian) at byte N*K/4, then
+ *   28 zero bytes.
+ * [I2S] "I2_S NEON kernel for the canonical layout", "llama-quantize I2_S emits the
+ * canonical layout"; rows divisible by 128 per "Known gaps".  The trailer is used as
+ * scratch during the call.  Errors: NULL, SHAPE (K % 128 != 0, N or K <= 0), ALIGN. */
+bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                              bitnet_stream s);
+
+/* BitNetRMSNorm + per-token absmax int8 quantisation of x [T, K] (bf16 or fp32).
+ *   with gain:  ms = mean(x^2) (exact fixed-point sum, rounded once to fp32),
+ *               inv = 1 / sqrt(ms + eps),  y = (x * inv) * gain      (fp32, no FMA)
+ *   gain NULL:  y = x   (use_rms_norm off)
+ *   s_x[t] = 127 / max(max|y|, 1e-5);  q = clamp(round_half_even(y * s_x), -128, 127);
+ *   sum_q[t] = sum_k q[t, k]  (the activation sum the I2_S product subtracts)
+ * [RMS] use_rms_norm / rms_norm_eps; [IQ1] 8-bit activations.
+ * Outputs: q int8 [T, K], s_x fp32 [T], sum_q int32 [T].  1 <= K <= BITNET_MAX_K.
+ * Errors: NULL, SHAPE, ALIGN, DTYPE. */
+bitnet_status bitnet_rmsnorm_quant_act(const void* x, bitnet_dtype xt, const float* gain,
+                                       float eps, int64_t T, int64_t K, int8_t* q,
+                                       float* s_x, int32_t* sum_q, bitnet_stream s);
+
+/* One BitLinear product after bitnet_rmsnorm_quant_act:
+ *   acc[t, n] = sum_k q[t, k] * c[n, k] - sum_q[t]        (int32, = sum_k q * w exactly)
+ *   out[t, n] = fp32(acc) * (beta / s_x[t])               (beta from the packed trailer)
+ * written as bf16 (round to nearest even) or fp32 into out [T, N].  If acc_debug is not
+ * NULL the int32 accumulators are also written there ([T, N]).  [I2S] "I2_S NEON kernel
+ * for the canonical layout" (codes c = w + 1, activation-sum correction).
+ * Requires K % 128 == 0.  Errors: NULL, SHAPE, ALIGN, DTYPE. */
+bitnet_status bitnet_bitlinear(const int8_t* q, const float* s_x, const int32_t* sum_q,
+                               const uint8_t* packed, int64_t T, int64_t N, int64_t K,
+                               void* out, bitnet_dtype ot, int32_t* acc_debug,
+                               bitnet_stream s);
+
+/* Several BitLinears that share one quantised input (the q, k, v projections of a
+ * decoder block) in one launch.  `packed`, `N` and `out` are HOST arrays of n_tensors
+ * (1..4) entries; each tensor keeps its own scale.  Same arithmetic and errors as
+ * bitnet_bitlinear. */
+bitnet_status bitnet_bitlinear_group(const int8_t* q, const float* s_x, const int32_t* sum_q,
+                                     int n_tensors, const uint8_t* const* packed,
+                                     const int64_t* N, int64_t T, int64_t K,
+                                     void* const* out, bitnet_dtype ot, bitnet_stream s);
+
+/* The gate/up half of the BitNet FFN with its activation fused into the epilogue:
+ *   g = BitLinear(p_gate), u = BitLinear(p_up) on the same quantised input (fp32, internal)
+ *   h[t, i] = act(g) * u   (relu2 or SiLU exactly as in bitnet_ffn_block)
+ * p_gate, p_up: I2_S [I, K]; h: fp32 [T, I].  [RMS] BitNetMLP.forward (act_fn(gate_proj(x))
+ * * up_proj(x)); [I2S] "bitnet-b1.58: squared-ReLU FFN".  Errors as bitnet_bitlinear. */
+bitnet_status bitnet_bitlinear_gate_up_act(const int8_t* q, const float* s_x, const int32_t* sum_q,
+                                           const uint8_t* p_gate, const uint8_t* p_up, int64_t T,
+                                           int64_t I, int64_t K, bitnet_act act, float* h,
+                                           bitnet_stream s);
+
+/* Workspace of bitnet_ffn_block, in bytes (0 if a size is invalid). */
+size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I);
+
+/* Byte offsets inside that workspace, so that a caller can read the intermediates after
+ * a call: off[0] q_x int8 [T,H], off[1] s_x fp32 [T], off[2] sum_x int32 [T],
+ * off[3] h fp32 [T,I], off[4] q_h int8 [T,I], off[5] s_h fp32 [T], off[6] sum_h int32 [T].
+ * `off` is a HOST array of 7 entries.  Returns BITNET_ERR_SHAPE on invalid sizes. */
+bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size_t* off);
+
+/* The BitNet FFN block on x [T, H]:
+ *   (q_x, s_x, sum_x) = rmsnorm_quant(x, g_ffn)                 (ffn_norm; NULL = off)
+ *   g = BitLinear(gate), u = BitLinear(up)                       (fp32 [T, I], internal)
+ *   h = act(g) * u:  relu2: r = max(g, 0), h = (r*r)*u;
+ *                    SiLU:  h = fp32(g / (1 + exp(-g))) * u, exp taken in fp64
+ *   (q_h, s_h, sum_h) = rmsnorm_quant(h, g_sub)                  (ffn_sub_norm)
+ *   out = BitLinear(down)                                        (bf16 or fp32 [T, H])
+ * [RMS] BitNetMLP.forward = down(ffn_sub_norm(act(gate(x)) * up(x)));
+ * [I2S] "bitnet-b1.58: squared-ReLU FFN" (relu2 vs SiLU from config).
+ * p_gate, p_up: I2_S [I, H]; p_down: I2_S [H, I]; H % 128 == 0 and I % 128 == 0.
+ * ws: device workspace of at least bitnet_ffn_workspace_bytes(T, H, I) bytes (16-byte
+ * aligned).  Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
+bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn,
+                               const uint8_t* p_gate, const uint8_t* p_up,
+                               const float* g_sub, const uint8_t* p_down,
+                               int64_t T, int64_t H, int64_t I, bitnet_act act, float eps,
+                               void* out, bitnet_dtype ot, void* ws, size_t ws_bytes,
+                               bitnet_stream s);
+
+/* Synchronises `s`, then reads and clears the device status word of the current
+ * device: BITNET_OK, or BITNET_ERR_TIMEOUT if a kernel gave up a bounded wait since
+ * the last read. */
+bitnet_status bitnet_get_device_status(bitnet_stream s);
+
+/* Static English text of a status code. */
+const char* bitnet_status_string(bitnet_status st);
+
+/* The CUDA error text of the last BITNET_ERR_CUDA on this thread ("" if none). */
+const char* bitnet_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITNET_B200_H */

@@ -1,0 +1,208 @@
+"""Python binding of libbitnet_b200.so: the BitNet b1.58 BitLinear forward on B200.
+
+Argument marshalling only -- every step of the arithmetic runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (the library allocates no device memory:
+outputs and workspaces are allocated here with torch and passed down); calls are
+enqueued on torch's current stream.  The library must have been built
+(``python -m ternary_bitlinear_quantized_b200.build``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "lib", "i2s_packed_bytes", "pack_i2s", "rmsnorm_quant_act", "bitlinear", "bitlinear_group", "bitlinear_gate_up_act",
+    "ffn_workspace_bytes", "ffn_workspace_offsets", "ffn_block", "device_status", "BitnetError",
+    "BF16", "F32", "RELU2", "SILU",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+
+BF16, F32 = 0, 1
+RELU2, SILU = 0, 1
+_STATUS = {0: "ok", 1: "null pointer", 2: "invalid shape", 3: "pointer not 16-byte aligned",
+           4: "invalid dtype or activation", 5: "workspace missing or too small", 6: "CUDA error",
+           7: "kernel wait timed out"}
+
+EXPORTS = [
+    "bitnet_i2s_packed_bytes", "bitnet_pack_i2s", "bitnet_rmsnorm_quant_act", "bitnet_bitlinear",
+    "bitnet_bitlinear_group", "bitnet_bitlinear_gate_up_act", "bitnet_ffn_workspace_bytes", "bitnet_ffn_workspace_offsets",
+    "bitnet_ffn_block", "bitnet_get_device_status", "bitnet_status_string", "bitnet_last_error",
+]
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {_STATUS.get(status, status)}"
+        if status == 6:
+            msg += f" ({_lib.bitnet_last_error().decode()})"
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ternary_bitlinear_quantized_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    c_p, c_i64, c_i, c_f, c_sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "bitnet_i2s_packed_bytes": (c_sz, [c_i64, c_i64]),
+        "bitnet_pack_i2s": (c_i, [c_p, c_i64, c_i64, c_p, c_p]),
+        "bitnet_rmsnorm_quant_act": (c_i, [c_p, c_i, c_p, c_f, c_i64, c_i64, c_p, c_p, c_p, c_p]),
+        "bitnet_bitlinear": (c_i, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i, c_p, c_p]),
+        "bitnet_bitlinear_group": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_i64, c_i64, c_p, c_i, c_p]),
+        "bitnet_bitlinear_gate_up_act": (c_i, [c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_p, c_p]),
+        "bitnet_ffn_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
+        "bitnet_ffn_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_p]),
+        "bitnet_ffn_block": (c_i, [c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_i,
+                                   c_p, c_sz, c_p]),
+        "bitnet_get_device_status": (c_i, [c_p]),
+        "bitnet_status_string": (ctypes.c_char_p, [c_i]),
+        "bitnet_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise BitnetError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _torch_dtype(code: int) -> torch.dtype:
+    return torch.bfloat16 if code == BF16 else torch.float32
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# ----------------------------------------------------------------------------- API
+
+def i2s_packed_bytes(N: int, K: int) -> int:
+    return int(lib().bitnet_i2s_packed_bytes(N, K))
+
+
+def pack_i2s(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Latent fp32 weights [N, K] -> I2_S bytes (uint8 [N*K/4 + 32])."""
+    _need(W, "W")
+    N, K = W.shape
+    nbytes = i2s_packed_bytes(N, K)
+    if nbytes == 0:
+        raise BitnetError(2, "pack_i2s")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check(lib().bitnet_pack_i2s(_ptr(W), N, K, _ptr(out), _stream(stream)), "pack_i2s")
+    return out
+
+
+def rmsnorm_quant_act(x: torch.Tensor, gain: torch.Tensor | None, eps: float = 1e-6, out=None, stream=None):
+    """x bf16/fp32 [T, K] -> (q int8 [T, K], s_x fp32 [T], sum_q int32 [T])."""
+    _need(x, "x")
+    T, K = x.shape
+    if out is None:
+        out = (torch.empty(T, K, dtype=torch.int8, device=x.device),
+               torch.empty(T, dtype=torch.float32, device=x.device),
+               torch.empty(T, dtype=torch.int32, device=x.device))
+    q, s, sq = out
+    _check(lib().bitnet_rmsnorm_quant_act(_ptr(x), _dtype_code(x.dtype), _ptr(gain), eps, T, K, _ptr(q), _ptr(s),
+                                          _ptr(sq), _stream(stream)), "rmsnorm_quant_act")
+    return q, s, sq
+
+
+def bitlinear(q, s_x, sum_q, packed, N: int, out_dtype=torch.bfloat16, out=None, acc_debug=None, stream=None):
+    """acc = sum q*c - sum_q; out = fp32(acc) * (beta / s_x) as out_dtype [T, N]."""
+    T, K = q.shape
+    if out is None:
+        out = torch.empty(T, N, dtype=out_dtype, device=q.device)
+    _check(lib().bitnet_bitlinear(_ptr(q), _ptr(s_x), _ptr(sum_q), _ptr(packed), T, N, K, _ptr(out),
+                                  _dtype_code(out.dtype), _ptr(acc_debug), _stream(stream)), "bitlinear")
+    return out
+
+
+def bitlinear_group(q, s_x, sum_q, packed: list, Ns: list, out_dtype=torch.bfloat16, outs=None, stream=None):
+    """Several BitLinears sharing one quantised input, in one launch."""
+    T, K = q.shape
+    n = len(packed)
+    if outs is None:
+        outs = [torch.empty(T, N, dtype=out_dtype, device=q.device) for N in Ns]
+    P = (ctypes.c_void_p * n)(*[p.data_ptr() for p in packed])
+    NN = (ctypes.c_int64 * n)(*Ns)
+    O = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    _check(lib().bitnet_bitlinear_group(_ptr(q), _ptr(s_x), _ptr(sum_q), n, ctypes.cast(P, ctypes.c_void_p),
+                                        ctypes.cast(NN, ctypes.c_void_p), T, K, ctypes.cast(O, ctypes.c_void_p),
+                                        _dtype_code(outs[0].dtype), _stream(stream)), "bitlinear_group")
+    return outs
+
+
+def bitlinear_gate_up_act(q, s_x, sum_q, p_gate, p_up, I: int, act: int = RELU2, out=None, stream=None):
+    """h = act(gate) * up, fp32 [T, I], from one quantised input (the FFN's first half)."""
+    T, K = q.shape
+    if out is None:
+        out = torch.empty(T, I, dtype=torch.float32, device=q.device)
+    _check(lib().bitnet_bitlinear_gate_up_act(_ptr(q), _ptr(s_x), _ptr(sum_q), _ptr(p_gate), _ptr(p_up), T, I, K,
+                                              act, _ptr(out), _stream(stream)), "bitlinear_gate_up_act")
+    return out
+
+
+def ffn_workspace_bytes(T: int, H: int, I: int) -> int:
+    return int(lib().bitnet_ffn_workspace_bytes(T, H, I))
+
+
+def ffn_workspace_offsets(T: int, H: int, I: int) -> list[int]:
+    off = (ctypes.c_size_t * 7)()
+    _check(lib().bitnet_ffn_workspace_offsets(T, H, I, ctypes.cast(off, ctypes.c_void_p)), "ffn_workspace_offsets")
+    return list(off)
+
+
+def ffn_block(x, g_ffn, p_gate, p_up, g_sub, p_down, I: int, act: int = RELU2, eps: float = 1e-6,
+              out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+    """BitNet FFN: down(ffn_sub_norm(act(gate(x)) * up(x))) on x [T, H]."""
+    _need(x, "x")
+    T, H = x.shape
+    if out is None:
+        out = torch.empty(T, H, dtype=out_dtype, device=x.device)
+    nws = ffn_workspace_bytes(T, H, I)
+    if ws is None:
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().bitnet_ffn_block(_ptr(x), _dtype_code(x.dtype), _ptr(g_ffn), _ptr(p_gate), _ptr(p_up), _ptr(g_sub),
+                                  _ptr(p_down), T, H, I, act, eps, _ptr(out), _dtype_code(out.dtype), _ptr(ws),
+                                  ws.numel(), _stream(stream)), "ffn_block")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word (0 = ok, 7 = a wait timed out)."""
+    return int(lib().bitnet_get_device_status(_stream(stream)))

@@ -1,0 +1,328 @@
+// The C ABI of include/bitnet_b200.h: argument checks, launch configuration and the
+// order of launches on the caller's stream.  Every step of the arithmetic runs in the
+// kernels of quant.cuh, pack.cuh, gemv.cuh and gemm_tc.cuh (one translation unit, so
+// that the device status word needs no relocatable device code).
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "quant.cuh"
+#include "pack.cuh"
+#include "gemv.cuh"
+
+namespace bitnet {
+
+static thread_local std::string t_last_error;
+
+static bitnet_status cuda_fail(cudaError_t e, const char* where) {
+  t_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return BITNET_ERR_CUDA;
+}
+
+#define BN_CUDA(call, where)                        \
+  do {                                              \
+    cudaError_t _e = (call);                        \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launch with programmatic stream serialisation: the kernel may begin while the
+// previous kernel on the stream is still running; it calls griddepcontrol.wait before
+// reading anything that kernel produced.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+static int device_sm_count() {
+  static thread_local int cached_dev = -1, cached_sms = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != cached_dev) {
+    cudaDeviceGetAttribute(&cached_sms, cudaDevAttrMultiProcessorCount, dev);
+    cached_dev = dev;
+  }
+  return cached_sms > 0 ? cached_sms : 148;
+}
+
+// ------------------------------------------------------------------ quant
+static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T, int64_t K,
+                                   int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
+  if (T == 0) return BITNET_OK;
+  int threads = (int)((K / 8 + 31) / 32 * 32);
+  threads = threads < 128 ? 128 : (threads > 1024 ? 1024 : threads);
+  const size_t smem = (size_t)K * sizeof(float);
+  const size_t esz = xt == BITNET_BF16 ? 2 : 4;
+  const int vec = (K % 8 == 0) && aligned16(x) && aligned16(q) && ((K * esz) % 16 == 0);
+  cudaError_t e;
+  if (smem > 48 * 1024) {
+    // Opt in to the large dynamic shared memory once per device and kernel.
+    static int done_mask[2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int& done = done_mask[xt == BITNET_BF16 ? 0 : 1][dev & 63];
+    if (!done) {
+      e = xt == BITNET_BF16 ? cudaFuncSetAttribute(k_rmsnorm_quant<__nv_bfloat16>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, BITNET_MAX_K * 4)
+                            : cudaFuncSetAttribute(k_rmsnorm_quant<float>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, BITNET_MAX_K * 4);
+      if (e != cudaSuccess) return cuda_fail(e, "quant attribute");
+      done = 1;
+    }
+  }
+  if (xt == BITNET_BF16) {
+    e = launch(k_rmsnorm_quant<__nv_bfloat16>, dim3((unsigned)T), dim3(threads), smem, s, true,
+               reinterpret_cast<const __nv_bfloat16*>(x), gain, eps, (int)K, q, s_x, sum_q, vec);
+  } else {
+    e = launch(k_rmsnorm_quant<float>, dim3((unsigned)T), dim3(threads), smem, s, true,
+               reinterpret_cast<const float*>(x), gain, eps, (int)K, q, s_x, sum_q, vec);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "k_rmsnorm_quant");
+  return BITNET_OK;
+}
+
+// ------------------------------------------------------------------ product
+static bitnet_status enqueue_gemv(const int8_t* q, const float* s_x, const int32_t* sum_q, int n_tensors,
+                                  const uint8_t* const* packed, const int64_t* N, void* const* out,
+                                  int32_t* const* acc_debug, int64_t T, int64_t K, bitnet_dtype ot,
+                                  bool ffn, bitnet_act act, float* h, cudaStream_t s) {
+  if (T == 0) return BITNET_OK;
+  GemvArgs a = {};
+  a.q = q;
+  a.s_x = s_x;
+  a.sum_q = sum_q;
+  a.T = (int)T;
+  a.K = (int)K;
+  a.n_tensors = n_tensors;
+  a.out_dtype = ot;
+  a.act = act;
+  a.h = h;
+  int tiles = 0;
+  for (int i = 0; i < n_tensors; ++i) {
+    a.t[i].packed = packed[i];
+    a.t[i].out = out ? out[i] : nullptr;
+    a.t[i].acc_debug = acc_debug ? acc_debug[i] : nullptr;
+    a.t[i].N = (int)N[i];
+    a.t[i].tile_begin = tiles;
+    if (!ffn || i == 0) tiles += (int)((N[i] + GEMV_ROWS - 1) / GEMV_ROWS);
+  }
+  a.n_tiles = tiles;
+  cudaError_t e = ffn ? launch(k_gemv_mma<true>, dim3(tiles), dim3(GEMV_WARPS * 32), 0, s, true, a)
+                      : launch(k_gemv_mma<false>, dim3(tiles), dim3(GEMV_WARPS * 32), 0, s, true, a);
+  if (e != cudaSuccess) return cuda_fail(e, "k_gemv_mma");
+  return BITNET_OK;
+}
+
+}  // namespace bitnet
+
+using namespace bitnet;
+
+// ====================================================================== C ABI
+extern "C" {
+
+size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  return (size_t)(N * K / 4 + 32);
+}
+
+bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* packed, bitnet_stream stream) {
+  if (!W || !packed) return BITNET_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % 128 != 0 || N * K >= (1ll << 40)) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed)) return BITNET_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n = N * K;
+  PackScratch* sc = reinterpret_cast<PackScratch*>(packed + n / 4);
+  const int sms = device_sm_count();
+  long long want = (n / 4 + 255) / 256;
+  const unsigned grid = (unsigned)(want < sms * 8 ? want : sms * 8);
+  long long wantc = (n / 16 + 255) / 256;
+  const unsigned gridc = (unsigned)(wantc < sms * 16 ? wantc : sms * 16);
+  cudaError_t e;
+  if ((e = launch(k_pack_clear, dim3(1), dim3(1), 0, s, false, sc)) != cudaSuccess) return cuda_fail(e, "k_pack_clear");
+  if ((e = launch(k_pack_absmax, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
+    return cuda_fail(e, "k_pack_absmax");
+  if ((e = launch(k_pack_sum, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
+    return cuda_fail(e, "k_pack_sum");
+  if ((e = launch(k_pack_codes, dim3(gridc), dim3(256), 0, s, false, W, n, (const PackScratch*)sc,
+                  reinterpret_cast<uint32_t*>(packed))) != cudaSuccess)
+    return cuda_fail(e, "k_pack_codes");
+  if ((e = launch(k_pack_trailer, dim3(1), dim3(1), 0, s, false, sc, n)) != cudaSuccess)
+    return cuda_fail(e, "k_pack_trailer");
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_rmsnorm_quant_act(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T,
+                                       int64_t K, int8_t* q, float* s_x, int32_t* sum_q, bitnet_stream stream) {
+  if (xt != BITNET_BF16 && xt != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (T < 0 || K <= 0 || K > BITNET_MAX_K || T > 0x7FFFFFFFll) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!x || !q || !s_x || !sum_q) return BITNET_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(s_x) || !aligned16(sum_q) || (gain && !aligned16(gain)))
+    return BITNET_ERR_ALIGN;
+  return enqueue_quant(x, xt, gain, eps, T, K, q, s_x, sum_q, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static bitnet_status check_product_args(const int8_t* q, const float* s_x, const int32_t* sum_q, int64_t T,
+                                        int64_t K, bitnet_dtype ot) {
+  if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (T < 0 || K <= 0 || K % 128 != 0 || K > BITNET_MAX_K || T > 0x7FFFFFFFll) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!q || !s_x || !sum_q) return BITNET_ERR_NULL;
+  if (!aligned16(q) || !aligned16(s_x) || !aligned16(sum_q)) return BITNET_ERR_ALIGN;
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_bitlinear(const int8_t* q, const float* s_x, const int32_t* sum_q, const uint8_t* packed,
+                               int64_t T, int64_t N, int64_t K, void* out, bitnet_dtype ot, int32_t* acc_debug,
+                               bitnet_stream stream) {
+  bitnet_status st = check_product_args(q, s_x, sum_q, T, K, ot);
+  if (st != BITNET_OK) return st;
+  if (N <= 0 || N > (1 << 30)) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!packed || !out) return BITNET_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(out) || (acc_debug && !aligned16(acc_debug))) return BITNET_ERR_ALIGN;
+  const uint8_t* p[1] = {packed};
+  const int64_t n[1] = {N};
+  void* o[1] = {out};
+  int32_t* d[1] = {acc_debug};
+  return enqueue_gemv(q, s_x, sum_q, 1, p, n, o, d, T, K, ot, false, BITNET_RELU2, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_bitlinear_group(const int8_t* q, const float* s_x, const int32_t* sum_q, int n_tensors,
+                                     const uint8_t* const* packed, const int64_t* N, int64_t T, int64_t K,
+                                     void* const* out, bitnet_dtype ot, bitnet_stream stream) {
+  bitnet_status st = check_product_args(q, s_x, sum_q, T, K, ot);
+  if (st != BITNET_OK) return st;
+  if (n_tensors < 1 || n_tensors > 4) return BITNET_ERR_SHAPE;
+  if (!packed || !N || !out) return BITNET_ERR_NULL;
+  for (int i = 0; i < n_tensors; ++i) {
+    if (N[i] <= 0 || N[i] > (1 << 30)) return BITNET_ERR_SHAPE;
+    if (T > 0 && (!packed[i] || !out[i])) return BITNET_ERR_NULL;
+    if (T > 0 && (!aligned16(packed[i]) || !aligned16(out[i]))) return BITNET_ERR_ALIGN;
+  }
+  if (T == 0) return BITNET_OK;
+  return enqueue_gemv(q, s_x, sum_q, n_tensors, packed, N, out, nullptr, T, K, ot, false, BITNET_RELU2, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_bitlinear_gate_up_act(const int8_t* q, const float* s_x, const int32_t* sum_q,
+                                           const uint8_t* p_gate, const uint8_t* p_up, int64_t T, int64_t I,
+                                           int64_t K, bitnet_act act, float* h, bitnet_stream stream) {
+  bitnet_status st = check_product_args(q, s_x, sum_q, T, K, BITNET_F32);
+  if (st != BITNET_OK) return st;
+  if (act != BITNET_RELU2 && act != BITNET_SILU) return BITNET_ERR_DTYPE;
+  if (I <= 0 || I > (1 << 30)) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!p_gate || !p_up || !h) return BITNET_ERR_NULL;
+  if (!aligned16(p_gate) || !aligned16(p_up) || !aligned16(h)) return BITNET_ERR_ALIGN;
+  const uint8_t* gu[2] = {p_gate, p_up};
+  const int64_t nI[2] = {I, I};
+  return enqueue_gemv(q, s_x, sum_q, 2, gu, nI, nullptr, nullptr, T, K, BITNET_F32, true, act, h,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+static size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size_t* off) {
+  if (!off) return BITNET_ERR_NULL;
+  if (T < 0 || H <= 0 || I <= 0) return BITNET_ERR_SHAPE;
+  size_t o = 0;
+  off[0] = o; o = align_up(o + (size_t)T * H);      // q_x
+  off[1] = o; o = align_up(o + (size_t)T * 4);      // s_x
+  off[2] = o; o = align_up(o + (size_t)T * 4);      // sum_x
+  off[3] = o; o = align_up(o + (size_t)T * I * 4);  // h
+  off[4] = o; o = align_up(o + (size_t)T * I);      // q_h
+  off[5] = o; o = align_up(o + (size_t)T * 4);      // s_h
+  off[6] = o; o = align_up(o + (size_t)T * 4);      // sum_h
+  return BITNET_OK;
+}
+
+size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I) {
+  size_t off[7];
+  if (bitnet_ffn_workspace_offsets(T, H, I, off) != BITNET_OK) return 0;
+  return align_up(off[6] + (size_t)T * 4);
+}
+
+bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
+                               const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T, int64_t H,
+                               int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot, void* ws,
+                               size_t ws_bytes, bitnet_stream stream) {
+  if (xt != BITNET_BF16 && xt != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (act != BITNET_RELU2 && act != BITNET_SILU) return BITNET_ERR_DTYPE;
+  if (T < 0 || T > 0x7FFFFFFFll || H <= 0 || I <= 0 || H % 128 || I % 128 || H > BITNET_MAX_K || I > BITNET_MAX_K)
+    return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!x || !p_gate || !p_up || !p_down || !out) return BITNET_ERR_NULL;
+  if (!ws) return BITNET_ERR_WORKSPACE;
+  if (ws_bytes < bitnet_ffn_workspace_bytes(T, H, I)) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(p_gate) || !aligned16(p_up) || !aligned16(p_down) || !aligned16(out) ||
+      !aligned16(ws) || (g_ffn && !aligned16(g_ffn)) || (g_sub && !aligned16(g_sub)))
+    return BITNET_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  size_t off[7];
+  bitnet_ffn_workspace_offsets(T, H, I, off);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  int8_t* q_x = reinterpret_cast<int8_t*>(w + off[0]);
+  float* s_x = reinterpret_cast<float*>(w + off[1]);
+  int32_t* sum_x = reinterpret_cast<int32_t*>(w + off[2]);
+  float* h = reinterpret_cast<float*>(w + off[3]);
+  int8_t* q_h = reinterpret_cast<int8_t*>(w + off[4]);
+  float* s_h = reinterpret_cast<float*>(w + off[5]);
+  int32_t* sum_h = reinterpret_cast<int32_t*>(w + off[6]);
+
+  bitnet_status st = enqueue_quant(x, xt, g_ffn, eps, T, H, q_x, s_x, sum_x, s);
+  if (st != BITNET_OK) return st;
+  const uint8_t* gu[2] = {p_gate, p_up};
+  const int64_t nI[2] = {I, I};
+  st = enqueue_gemv(q_x, s_x, sum_x, 2, gu, nI, nullptr, nullptr, T, H, BITNET_F32, true, act, h, s);
+  if (st != BITNET_OK) return st;
+  st = enqueue_quant(h, BITNET_F32, g_sub, eps, T, I, q_h, s_h, sum_h, s);
+  if (st != BITNET_OK) return st;
+  const uint8_t* pd[1] = {p_down};
+  const int64_t nH[1] = {H};
+  void* o[1] = {out};
+  return enqueue_gemv(q_h, s_h, sum_h, 1, pd, nH, o, nullptr, T, I, ot, false, act, nullptr, s);
+}
+
+bitnet_status bitnet_get_device_status(bitnet_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  const int zero = 0;
+  BN_CUDA(cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s), "status read");
+  BN_CUDA(cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s), "status clear");
+  BN_CUDA(cudaStreamSynchronize(s), "status sync");
+  return v == 0 ? BITNET_OK : (bitnet_status)v;
+}
+
+const char* bitnet_status_string(bitnet_status st) {
+  switch (st) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_NULL: return "null pointer";
+    case BITNET_ERR_SHAPE: return "invalid shape";
+    case BITNET_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case BITNET_ERR_DTYPE: return "invalid dtype or activation";
+    case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+    case BITNET_ERR_CUDA: return "CUDA error";
+    case BITNET_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* bitnet_last_error(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// Shared device helpers of the sm_100a kernels: exact fp32/fp64 steps, block
+// reductions, programmatic-dependent-launch control, bulk L2 prefetch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/bitnet_b200.h"
+
+#define BN_DEV __device__ __forceinline__
+
+namespace bitnet {
+
+// Device status word (bounded waits that gave up set BITNET_ERR_TIMEOUT here).  The
+// library is one translation unit (bitnet_b200.cu includes every kernel header).
+__device__ int g_device_status = 0;
+
+// ---------------------------------------------------------------- launch control
+// Programmatic dependent launch: let the next kernel on the stream start its
+// prologue now; wait for the previous kernel's memory before reading activations.
+BN_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+BN_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Bulk prefetch of a contiguous global range into L2 (address and size 16-byte multiples).
+BN_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+BN_DEV uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ---------------------------------------------------------------- exact helpers
+// 2**e as an fp64 (exact for -1022 <= e <= 1023).
+BN_DEV double pow2_f64(int e) { return __longlong_as_double((long long)(1023 + e) << 52); }
+
+// E with M = m * 2**E, 0.5 <= m < 1, for a normal positive fp64 M.
+BN_DEV int frexp_exponent(double M) { return (int)((__double_as_longlong(M) >> 52) & 0x7FF) - 1022; }
+
+// Smallest L with 2**L >= n (n >= 1).
+BN_DEV int ceil_log2_i64(long long n) { return n <= 1 ? 0 : 64 - __clzll(n - 1); }
+
+// Fixed-point grid exponent e = 62 - E(M) - ceil_log2(n) of an order-free sum of n
+// non-negative terms whose maximum is M > 0.
+BN_DEV int fixed_point_exponent(double M, long long n) { return 62 - frexp_exponent(M) - ceil_log2_i64(n); }
+
+// fp32( (fp64(S) * 2**-e) / n ): the mean of a fixed-point sum.
+BN_DEV float fixed_point_mean(long long S, int e, long long n) {
+  if (S == 0) return 0.0f;
+  double v = __dmul_rn(__ll2double_rn(S), pow2_f64(-e));
+  return __double2float_rn(__ddiv_rn(v, __ll2double_rn(n)));
+}
+
+BN_DEV float bf16_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+
+// ---------------------------------------------------------------- reductions
+BN_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+BN_DEV long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+BN_DEV int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Block-wide reductions through a small shared scratch of >= 32 entries; every thread
+// gets the result.  max over non-negative floats and integer sums are exact, so the
+// result does not depend on the order.
+template <typename T, typename Op>
+BN_DEV T block_reduce(T v, T* scratch, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();  // scratch may still be read by a previous reduction
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  T r = scratch[0];
+  for (int w = 1; w < nw; ++w) r = op(r, scratch[w]);
+  return r;
+}
+
+struct MaxOp {
+  BN_DEV float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct AddOpLL {
+  BN_DEV long long operator()(long long a, long long b) const { return a + b; }
+};
+struct AddOpI {
+  BN_DEV int operator()(int a, int b) const { return a + b; }
+};
+
+}  // namespace bitnet

@@ -1,0 +1,156 @@
+// K-quant: fused BitNetRMSNorm + per-token absmax + int8 quantisation.
+//
+// "Add optional RMSNorm support to BitNet quantization (config + layers)": BitLinear
+// applies BitNetRMSNorm (eps 1e-6 by default) to the activations before they are
+// quantised; with use_rms_norm off (gain == nullptr) the activations go straight to
+// the absmax quantiser.  "More BitNet-like IQ1_S quantizations": the activations of
+// BitNet b1.58 are 8-bit.
+//
+// One CTA per token.  The row is staged once in shared memory as fp32; the three
+// reductions (max|x|, the fixed-point sum of x^2, max|y|) and the sum of q are exact,
+// so the result is independent of the thread count and of the order of summation.
+#pragma once
+#include "common.cuh"
+
+namespace bitnet {
+
+template <typename TIn>
+struct RowLoader;
+
+template <>
+struct RowLoader<__nv_bfloat16> {
+  static constexpr int V = 8;  // elements per 16-byte vector
+  BN_DEV static void load(const __nv_bfloat16* p, float* o) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  BN_DEV static float load1(const __nv_bfloat16* p) { return bf16_to_f32(*reinterpret_cast<const uint16_t*>(p)); }
+};
+
+template <>
+struct RowLoader<float> {
+  static constexpr int V = 8;
+  BN_DEV static void load(const float* p, float* o) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+  BN_DEV static float load1(const float* p) { return *p; }
+};
+
+// Quantise one staged row xs[0..K) in place of nothing: writes q, s_x, sum_q of the row.
+// `vec` says whether K % 8 == 0 and the row pointers are 16-byte aligned.
+BN_DEV void quantise_staged_row(float* xs, int K, const float* gain, float eps, int8_t* qrow,
+                                float* s_out, int32_t* sum_out, bool vec, void* red_scratch,
+                                float amax_x) {
+  float* redf = reinterpret_cast<float*>(red_scratch);
+  long long* redl = reinterpret_cast<long long*>(red_scratch);
+  int* redi = reinterpret_cast<int*>(red_scratch);
+  const int tid = threadIdx.x, nt = blockDim.x;
+
+  float a;
+  if (gain != nullptr) {
+    float ms = 0.0f;
+    if (amax_x > 0.0f) {
+      const double M = __dmul_rn((double)amax_x, (double)amax_x);
+      const int e = fixed_point_exponent(M, K);
+      const double p2e = pow2_f64(e);
+      long long part = 0;
+      for (int k = tid; k < K; k += nt) {
+        const double v = (double)xs[k];
+        part += __double2ll_rn(__dmul_rn(__dmul_rn(v, v), p2e));
+      }
+      const long long S = block_reduce(part, redl, AddOpLL());
+      ms = fixed_point_mean(S, e, K);
+    }
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    float am = 0.0f;
+    for (int k = tid; k < K; k += nt) {
+      const float y = __fmul_rn(__fmul_rn(xs[k], inv), __ldg(gain + k));
+      xs[k] = y;
+      am = fmaxf(am, fabsf(y));
+    }
+    a = block_reduce(am, redf, MaxOp());
+  } else {
+    a = amax_x;  // y = x
+  }
+  const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+  int sum = 0;
+  if (vec) {
+    for (int k = tid * 8; k < K; k += nt * 8) {
+      uint32_t w[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int v = __float2int_rn(__fmul_rn(xs[k + 4 * h + j], s));
+          v = min(127, max(-128, v));
+          sum += v;
+          packed |= (uint32_t)(v & 0xFF) << (8 * j);
+        }
+        w[h] = packed;
+      }
+      *reinterpret_cast<uint2*>(qrow + k) = make_uint2(w[0], w[1]);
+    }
+  } else {
+    for (int k = tid; k < K; k += nt) {
+      int v = __float2int_rn(__fmul_rn(xs[k], s));
+      v = min(127, max(-128, v));
+      sum += v;
+      qrow[k] = (int8_t)v;
+    }
+  }
+  sum = block_reduce(sum, redi, AddOpI());
+  if (tid == 0) {
+    *s_out = s;
+    *sum_out = sum;
+  }
+}
+
+// Stage row `x` [K] into xs as fp32; returns max|x| over the block.
+template <typename TIn>
+BN_DEV float stage_row(const TIn* x, int K, float* xs, bool vec, void* red_scratch) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  float am = 0.0f;
+  if (vec) {
+    for (int k = tid * 8; k < K; k += nt * 8) {
+      float v[8];
+      RowLoader<TIn>::load(x + k, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        xs[k + j] = v[j];
+        am = fmaxf(am, fabsf(v[j]));
+      }
+    }
+  } else {
+    for (int k = tid; k < K; k += nt) {
+      const float v = RowLoader<TIn>::load1(x + k);
+      xs[k] = v;
+      am = fmaxf(am, fabsf(v));
+    }
+  }
+  return block_reduce(am, reinterpret_cast<float*>(red_scratch), MaxOp());
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ x, const float* __restrict__ gain,
+                                                        float eps, int K, int8_t* __restrict__ q,
+                                                        float* __restrict__ s_x, int32_t* __restrict__ sum_q,
+                                                        int vec) {
+  extern __shared__ float xs[];
+  __shared__ long long red[32];
+  const long long t = blockIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  const float amax = stage_row<TIn>(x + t * K, K, xs, vec != 0, red);
+  quantise_staged_row(xs, K, gain, eps, q + t * K, s_x + t, sum_q + t, vec != 0, red, amax);
+}
+
+}  // namespace bitnet

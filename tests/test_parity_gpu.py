@@ -1,0 +1,186 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element, on the same
+seeded inputs.  Bytes, int8 activations, activation sums and int32 accumulators must be
+bit-exact; float outputs within 1e-3 (fp32) / 1e-2 (bf16) max relative error."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import ternary_bitlinear_quantized_b200 as tb
+import workloads
+from oracle import bitnet_oracle as O
+from tests.parity_util import act_to_np, assert_close, bf16_to_np, oracle_rows, out_to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    tb.lib()
+    yield
+    assert tb.device_status() == 0
+
+
+def gpu_pack(W: torch.Tensor) -> torch.Tensor:
+    return tb.pack_i2s(W.to(DEV).contiguous())
+
+
+# ----------------------------------------------------------------------------- a1: pack
+
+@pytest.mark.parametrize("N,K,seed", [(1, 128, 0), (17, 384, 1), (300, 640, 2), (1000, 2560, 3), (64, 6912, 4)])
+def test_pack_bytes_bitexact(N, K, seed):
+    W = workloads.latent_weight(N, K, seed, "pack")
+    got = gpu_pack(W).cpu().numpy()
+    ref = O.pack_i2s(W.numpy())
+    assert got.shape == ref.shape
+    assert np.array_equal(got, ref)
+
+
+def test_pack_special_cases():
+    zero = torch.zeros(2, 256)
+    assert np.array_equal(gpu_pack(zero).cpu().numpy(), O.pack_i2s(zero.numpy()))
+    k = np.arange(128)
+    hand = np.where(k % 3 == 0, 0.02, np.where(k % 3 == 1, -0.02, 0.0)).astype(np.float32).reshape(1, 128)
+    assert np.array_equal(gpu_pack(torch.from_numpy(hand)).cpu().numpy(), O.pack_i2s(hand))
+    rng = np.random.default_rng(5)
+    tern = (rng.integers(-1, 2, size=(33, 512)) * 0.0375).astype(np.float32)
+    got = gpu_pack(torch.from_numpy(tern)).cpu().numpy()
+    assert np.array_equal(got, O.pack_i2s(tern))
+    codes, _ = O.unpack_i2s(got, 33, 512)
+    assert np.array_equal(codes.astype(int) - 1, np.rint(tern / 0.0375).astype(int))
+
+
+def test_pack_repeatable_across_streams():
+    W = workloads.latent_weight(257, 1024, 9, "rep").to(DEV)
+    a = tb.pack_i2s(W)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = tb.pack_i2s(W)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------- a2: quant
+
+@pytest.mark.parametrize("T,K,dtype,use_gain,outliers", [
+    (1, 2560, torch.bfloat16, True, False),
+    (5, 640, torch.bfloat16, True, True),
+    (3, 6912, torch.float32, True, False),
+    (4, 2560, torch.bfloat16, False, False),
+    (2, 100, torch.bfloat16, True, False),     # K not a multiple of 8: scalar path
+    (3, 27648, torch.float32, True, False),
+    (2, 28672, torch.bfloat16, True, True),
+    (130, 384, torch.bfloat16, True, True),
+])
+def test_quant_bitexact(T, K, dtype, use_gain, outliers):
+    x = workloads.activations(T, K, 11, "quant", outliers)
+    if dtype == torch.float32:
+        x = x.float() * 3.0 + 0.25 * torch.randn(T, K, generator=torch.Generator().manual_seed(1))
+    x[T // 2] = 0  # a zero token
+    g = workloads.gain(K, 11, "quant") if use_gain else None
+    q, s, sq = tb.rmsnorm_quant_act(x.to(DEV), None if g is None else g.to(DEV), 1e-6)
+    rq, rs, rsq = O.rmsnorm_quant_act(act_to_np(x), None if g is None else g.numpy(), 1e-6)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(sq.cpu().numpy(), rsq)
+
+
+# ----------------------------------------------------------------------------- a3/a4: product
+
+def run_bitlinear(T, N, K, seed, out_dtype, outliers=False):
+    W = workloads.latent_weight(N, K, seed, "bl")
+    x = workloads.activations(T, K, seed, "bl", outliers)
+    g = workloads.gain(K, seed, "bl")
+    packed_ref = O.pack_i2s(W.numpy())
+    packed = torch.from_numpy(packed_ref).to(DEV)  # oracle bytes: this test isolates the product
+    q, s, sq = tb.rmsnorm_quant_act(x.to(DEV), g.to(DEV), 1e-6)
+    acc = torch.empty(T, N, dtype=torch.int32, device=DEV)
+    out = tb.bitlinear(q, s, sq, packed, N, out_dtype, acc_debug=acc)
+    rq, rs, rsq = O.rmsnorm_quant_act(bf16_to_np(x), g.numpy(), 1e-6)
+    dt = "bf16" if out_dtype == torch.bfloat16 else "f32"
+    ref, racc = O.bitlinear(rq, rs, rsq, packed_ref, N, K, dt, return_acc=True)
+    return out, acc, ref, racc, dt
+
+
+@pytest.mark.parametrize("T,N,K", [(1, 1, 128), (1, 300, 640), (3, 17, 384), (8, 2560, 2560), (9, 100, 1024),
+                                   (16, 64, 2560), (17, 48, 256), (33, 40, 640), (1, 640, 6912)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_bitlinear_parity(T, N, K, out_dtype):
+    out, acc, ref, racc, dt = run_bitlinear(T, N, K, T * 1000 + N, out_dtype)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    got = out_to_np(out)
+    assert_close(got, ref, dt)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))  # same op sequence: bit-identical
+
+
+def test_bitlinear_group_matches_singles():
+    T, K = 2, 2560
+    Ns = [2560, 640, 640]
+    x = workloads.activations(T, K, 3, "grp")
+    g = workloads.gain(K, 3, "grp")
+    Ws = [workloads.latent_weight(n, K, 3, f"grp{i}") for i, n in enumerate(Ns)]
+    packs_ref = [O.pack_i2s(W.numpy()) for W in Ws]
+    packs = [torch.from_numpy(p).to(DEV) for p in packs_ref]
+    q, s, sq = tb.rmsnorm_quant_act(x.to(DEV), g.to(DEV), 1e-6)
+    outs = tb.bitlinear_group(q, s, sq, packs, Ns, torch.bfloat16)
+    rq, rs, rsq = O.rmsnorm_quant_act(bf16_to_np(x), g.numpy(), 1e-6)
+    for o, p, n in zip(outs, packs_ref, Ns):
+        ref = O.bitlinear(rq, rs, rsq, p, n, K, "bf16")
+        assert np.array_equal(out_to_np(o), ref)
+
+
+# ----------------------------------------------------------------------------- a5-a7: FFN block
+
+def run_ffn(T, H, I, act, seed, out_dtype=torch.bfloat16, x_dtype=torch.bfloat16):
+    sh = workloads.BlockShape("ffn-test", hidden=H, n_q=H, n_kv=H, inter=I, act=act)
+    d = workloads.block_inputs(sh, T, seed, ffn_only=True)
+    x = d["x"] if x_dtype == torch.bfloat16 else d["x"].float()
+    pr = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in ("gate", "up", "down")}
+    pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
+    ws = torch.empty(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
+    code = tb.RELU2 if act == "relu2" else tb.SILU
+    out = tb.ffn_block(x.to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], d["g_ffn_sub_norm"].to(DEV),
+                       pg["down"], I, code, 1e-6, out_dtype, ws=ws)
+    dt = "bf16" if out_dtype == torch.bfloat16 else "f32"
+    ref, mid = O.ffn_block(act_to_np(x), d["g_ffn_norm"].numpy(), pr["gate"], pr["up"], d["g_ffn_sub_norm"].numpy(),
+                           pr["down"], H, I, act, 1e-6, dt, return_intermediates=True)
+    return out, ws, ref, mid, dt
+
+
+@pytest.mark.parametrize("act", ["relu2", "silu"])
+@pytest.mark.parametrize("T,H,I", [(1, 256, 384), (3, 640, 1280), (17, 256, 640)])
+def test_ffn_block_parity(act, T, H, I):
+    out, ws, ref, mid, dt = run_ffn(T, H, I, act, seed=T + H)
+    off = tb.ffn_workspace_offsets(T, H, I)
+    wsn = ws.cpu().numpy()
+    q_x = wsn[off[0]:off[0] + T * H].view(np.int8).reshape(T, H)
+    h = wsn[off[3]:off[3] + T * I * 4].view(np.float32).reshape(T, I)
+    q_h = wsn[off[4]:off[4] + T * I].view(np.int8).reshape(T, I)
+    sum_h = wsn[off[6]:off[6] + T * 4].view(np.int32)
+    assert np.array_equal(q_x, mid["q"])
+    assert np.array_equal(h.view(np.uint32), mid["h"].view(np.uint32))
+    assert np.array_equal(q_h, mid["q_h"])
+    assert np.array_equal(sum_h, mid["sum_h"])
+    got = out_to_np(out)
+    assert_close(got, ref, dt)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_ffn_block_fp32_io():
+    out, _, ref, _, dt = run_ffn(2, 384, 512, "silu", seed=5, out_dtype=torch.float32, x_dtype=torch.float32)
+    assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
+
+
+def test_empty_token_batch_is_noop():
+    q = torch.empty(0, 256, dtype=torch.int8, device=DEV)
+    s = torch.empty(0, dtype=torch.float32, device=DEV)
+    sq = torch.empty(0, dtype=torch.int32, device=DEV)
+    packed = gpu_pack(workloads.latent_weight(32, 256, 0, "e"))
+    out = tb.bitlinear(q, s, sq, packed, 32, torch.bfloat16)
+    assert out.shape == (0, 32)
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device=DEV)
+    qq, _, _ = tb.rmsnorm_quant_act(x, None)
+    assert qq.shape == (0, 256)
