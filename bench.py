@@ -297,6 +297,9 @@ def time_dominant(wl: Workload, launches: int):
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
     stream = torch.cuda.current_stream()
+    # Hold the GPU while the host enqueues, so that no host launch latency falls between
+    # an event pair; the events also keep consecutive launches from overlapping.
+    torch.cuda._sleep(int(launches * 60_000))
     for i, (a, b) in enumerate(evs):
         a.record(stream)
         fn(i % R)

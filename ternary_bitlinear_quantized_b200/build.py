@@ -36,7 +36,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         return LIB
     cmd = [nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "--fmad=false", "-Xcompiler", "-fPIC", "-shared",
            "-cudart", "static", "-I", os.path.join(os.path.dirname(HERE), "include"),
-           "-o", LIB + ".tmp", os.path.join(CSRC, "bitnet_b200.cu"), "-lcuda"]
+           "-o", LIB + ".tmp", os.path.join(CSRC, "bitnet_b200.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)

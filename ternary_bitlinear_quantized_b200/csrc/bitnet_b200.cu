@@ -10,6 +10,8 @@
 #include "quant.cuh"
 #include "pack.cuh"
 #include "gemv.cuh"
+#include "decode.cuh"
+#include "gemm_tc.cuh"
 
 namespace bitnet {
 
@@ -58,6 +60,54 @@ static int device_sm_count() {
   return cached_sms > 0 ? cached_sms : 148;
 }
 
+// Opt a kernel in to the full dynamic shared memory of the SM, once per device.
+static cudaError_t opt_in_smem(const void* kern, int slot) {
+  static int done[8][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& d = done[slot & 7][dev & 63];
+  if (d) return cudaSuccess;
+  int max_optin = 0;
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin - (int)fa.sharedSizeBytes);
+  if (e == cudaSuccess) d = 1;
+  return e;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows, cols] (row stride `stride` bytes) with a box of box_cols x box_rows.
+static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
+                        uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ quant
 static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T, int64_t K,
                                    int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
@@ -95,6 +145,61 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
 }
 
 // ------------------------------------------------------------------ product
+// Prefill: the tcgen05 kernel, from the same arguments as the decode kernel.
+static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s) {
+  const int NT = ffn ? 2 : 1;
+  TcArgs a = {};
+  a.s_x = g.s_x;
+  a.sum_q = g.sum_q;
+  a.T = g.T;
+  a.K = g.K;
+  int bn = (g.T + 15) / 16 * 16;
+  const int bn_max = ffn ? 128 : 256;
+  a.BN = bn > bn_max ? bn_max : bn;
+  a.n_tensors = g.n_tensors;
+  a.out_dtype = g.out_dtype;
+  a.act = g.act;
+  a.h = g.h;
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_map_u8(&maps.act, g.q, (uint64_t)g.K, (uint64_t)g.T, (uint64_t)g.K, TC_BK, (uint32_t)a.BN, true))
+    return cuda_fail(cudaErrorInvalidValue, "tensor map (activations)");
+  int mt = 0;
+  for (int i = 0; i < g.n_tensors; ++i) {
+    a.t[i].packed = g.t[i].packed;
+    a.t[i].out = g.t[i].out;
+    a.t[i].acc_debug = g.t[i].acc_debug;
+    a.t[i].N = g.t[i].N;
+    a.t[i].m_tile_begin = mt;
+    if (!ffn || i == 0) mt += (g.t[i].N + TC_BM - 1) / TC_BM;
+    if (!make_map_u8(&maps.w[i], g.t[i].packed, (uint64_t)(g.K / 4), (uint64_t)g.t[i].N, (uint64_t)(g.K / 4), 32,
+                     TC_BM, false))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map (weights)");
+  }
+  a.m_tiles = mt;
+  a.tok_tiles = (g.T + a.BN - 1) / a.BN;
+  const uint32_t stage_bytes = (uint32_t)((NT * TC_BM * TC_BK + a.BN * TC_BK + NT * TC_BM * 32 + 1023) / 1024 * 1024);
+  int dev = 0, max_optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa;
+  void (*kern)(const TcMaps, const TcArgs) = ffn ? k_gemm_tc<true> : k_gemm_tc<false>;
+  cudaError_t e = cudaFuncGetAttributes(&fa, (const void*)kern);
+  if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc attributes");
+  int stages = (int)((max_optin - (int)fa.sharedSizeBytes - 1024 - 256) / stage_bytes);
+  if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
+  if (stages < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_gemm_tc stages");
+  a.stages = stages;
+  const size_t smem = (size_t)stages * stage_bytes + 1024 + 256;
+  e = opt_in_smem((const void*)kern, 4 + (ffn ? 1 : 0));
+  if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc attribute");
+  const int total = a.m_tiles * a.tok_tiles;
+  const int sms = device_sm_count();
+  e = launch(kern, dim3(total < sms ? total : sms), dim3(TC_THREADS), smem, s, true, maps, a);
+  if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc");
+  return BITNET_OK;
+}
+
 static bitnet_status enqueue_gemv(const int8_t* q, const float* s_x, const int32_t* sum_q, int n_tensors,
                                   const uint8_t* const* packed, const int64_t* N, void* const* out,
                                   int32_t* const* acc_debug, int64_t T, int64_t K, bitnet_dtype ot,
@@ -120,10 +225,20 @@ static bitnet_status enqueue_gemv(const int8_t* q, const float* s_x, const int32
     if (!ffn || i == 0) tiles += (int)((N[i] + GEMV_ROWS - 1) / GEMV_ROWS);
   }
   a.n_tiles = tiles;
-  cudaError_t e = ffn ? launch(k_gemv_mma<true>, dim3(tiles), dim3(GEMV_WARPS * 32), 0, s, true, a)
-                      : launch(k_gemv_mma<false>, dim3(tiles), dim3(GEMV_WARPS * 32), 0, s, true, a);
-  if (e != cudaSuccess) return cuda_fail(e, "k_gemv_mma");
-  return BITNET_OK;
+  cudaError_t e;
+  if (T <= DEC_MAX_T) {
+    int grid = 0;
+    const DecPlan p = plan_decode(tiles, (int)K, ffn, device_sm_count(), &grid);
+    const int tg = T <= 8 ? 1 : 2;
+    void (*kern)(const GemvArgs, const DecPlan) =
+        ffn ? (tg == 1 ? k_decode<true, 1> : k_decode<true, 2>) : (tg == 1 ? k_decode<false, 1> : k_decode<false, 2>);
+    if ((e = opt_in_smem((const void*)kern, (ffn ? 2 : 0) + tg - 1)) != cudaSuccess)
+      return cuda_fail(e, "k_decode attribute");
+    e = launch(kern, dim3(grid), dim3(DEC_THREADS), (size_t)p.smem_bytes, s, true, a, p);
+    if (e != cudaSuccess) return cuda_fail(e, "k_decode");
+    return BITNET_OK;
+  }
+  return enqueue_gemm_tc(a, ffn, s);
 }
 
 }  // namespace bitnet

@@ -106,7 +106,9 @@ def run_bitlinear(T, N, K, seed, out_dtype, outliers=False):
 
 
 @pytest.mark.parametrize("T,N,K", [(1, 1, 128), (1, 300, 640), (3, 17, 384), (8, 2560, 2560), (9, 100, 1024),
-                                   (16, 64, 2560), (17, 48, 256), (33, 40, 640), (1, 640, 6912)])
+                                   (16, 64, 2560), (17, 48, 256), (33, 40, 640), (1, 640, 6912), (2, 48, 8192),
+                                   (4, 33, 28672), (1, 28672, 128), (12, 150, 1152),
+                                   (64, 300, 640), (200, 130, 1280), (300, 256, 256), (513, 384, 2560)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_bitlinear_parity(T, N, K, out_dtype):
     out, acc, ref, racc, dt = run_bitlinear(T, N, K, T * 1000 + N, out_dtype)
@@ -116,8 +118,9 @@ def test_bitlinear_parity(T, N, K, out_dtype):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))  # same op sequence: bit-identical
 
 
-def test_bitlinear_group_matches_singles():
-    T, K = 2, 2560
+@pytest.mark.parametrize("T", [2, 100])
+def test_bitlinear_group_matches_singles(T):
+    K = 2560
     Ns = [2560, 640, 640]
     x = workloads.activations(T, K, 3, "grp")
     g = workloads.gain(K, 3, "grp")
@@ -151,7 +154,8 @@ def run_ffn(T, H, I, act, seed, out_dtype=torch.bfloat16, x_dtype=torch.bfloat16
 
 
 @pytest.mark.parametrize("act", ["relu2", "silu"])
-@pytest.mark.parametrize("T,H,I", [(1, 256, 384), (3, 640, 1280), (17, 256, 640)])
+@pytest.mark.parametrize("T,H,I", [(1, 256, 384), (3, 640, 1280), (17, 256, 640), (2, 8192, 512), (10, 1152, 2304),
+                                   (64, 512, 768), (130, 384, 1280)])
 def test_ffn_block_parity(act, T, H, I):
     out, ws, ref, mid, dt = run_ffn(T, H, I, act, seed=T + H)
     off = tb.ffn_workspace_offsets(T, H, I)
