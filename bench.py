@@ -191,8 +191,14 @@ class Workload:
         else:
             self.inputs = [self.d["x"]]
         self.offn = e(T, H)
-        self.ws = torch.empty(self.tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=self.dev)
-        self.outputs = ([self.oq, self.ok_, self.ov, self.offn] if self.kind == "block" else [self.offn])
+        # Zeroed once: the decode engine's grid-barrier counters live in the workspace.
+        nws = (self.tb.block_workspace_bytes(T, H, sh.n_q, I) if self.kind == "block"
+               else self.tb.ffn_workspace_bytes(T, H, I))
+        self.ws = torch.zeros(nws, dtype=torch.uint8, device=self.dev)
+        self.outputs = ([self.oq, self.ok_, self.ov, self.oo, self.offn] if self.kind == "block" else [self.offn])
+        if self.kind == "block":
+            self.gains = {k[2:]: v for k, v in self.d.items() if k.startswith("g_")}
+            self.outs = {"q": self.oq, "k": self.ok_, "v": self.ov, "o": self.oo, "ffn": self.offn}
 
     def step(self, c: int):
         tb, p = self.tb, self.copies[c]
@@ -201,28 +207,34 @@ class Workload:
             tb.bitlinear(q, s, sq, p["w"], self.tensors["w"][0], out=self.out)
             return
         d, sh = self.d, self.shape
-        ffn_in = d["x"]
         if self.kind == "block":
-            q, s, sq = tb.rmsnorm_quant_act(d["x"], d["g_attn_norm"], workloads.EPS, out=self.qx)
-            tb.bitlinear_group(q, s, sq, [p["q"], p["k"], p["v"]], [sh.n_q, sh.n_kv, sh.n_kv],
-                               outs=[self.oq, self.ok_, self.ov])
-            q, s, sq = tb.rmsnorm_quant_act(d["attn_out"], d["g_attn_sub_norm"], workloads.EPS, out=self.qa)
-            tb.bitlinear(q, s, sq, p["o"], sh.hidden, out=self.oo)
-            ffn_in = self.oo
-        tb.ffn_block(ffn_in, d["g_ffn_norm"], p["gate"], p["up"], d["g_ffn_sub_norm"], p["down"], sh.inter,
+            tb.decoder_block(d["x"], d["attn_out"], self.gains, p, sh.n_kv, sh.inter, self.act, workloads.EPS,
+                             outs=self.outs, ws=self.ws)
+            return
+        tb.ffn_block(d["x"], d["g_ffn_norm"], p["gate"], p["up"], d["g_ffn_sub_norm"], p["down"], sh.inter,
                      self.act, workloads.EPS, out=self.offn, ws=self.ws)
 
     def launches_per_step(self) -> int:
-        return {"bitlinear": 2, "block": 8, "ffn": 4}[self.kind]
+        """Launches of this library's kernels per step (the decode engine runs a whole
+        block or FFN in one launch; prefill launches quant + tensor-core product per layer)."""
+        if self.kind == "bitlinear":
+            return 2
+        if self.T <= 16:
+            return 1
+        return 8 if self.kind == "block" else 4
 
     def dominant(self):
-        """(label, callable(c), bytes per launch, ops per launch) of the largest product kernel:
-        the FFN's gate/up launch (relu2/SiLU epilogue) or the single BitLinear."""
+        """(label, callable(c), bytes per launch, ops per launch) of the dominant kernel: at
+        decode the single engine launch of the whole step; at prefill the FFN's gate/up
+        tensor-core launch (relu2/SiLU epilogue); for one BitLinear its product kernel."""
         tb = self.tb
+        if self.kind != "bitlinear" and self.T <= 16:
+            label = "k_engine (decoder block, one launch)" if self.kind == "block" else "k_engine (FFN, one launch)"
+            return (label, lambda c: self.step(c), self.packed_bytes, self.ops_per_step)
         if self.kind == "bitlinear":
             N, K = self.tensors["w"]
             q, s, sq = self.qbuf
-            return ("k_gemv_mma (bitlinear)", lambda c: tb.bitlinear(q, s, sq, self.copies[c]["w"], N, out=self.out),
+            return ("k_engine (bitlinear)" if self.T <= 16 else "k_gemm_tc (bitlinear)", lambda c: tb.bitlinear(q, s, sq, self.copies[c]["w"], N, out=self.out),
                     tb.i2s_packed_bytes(N, K), 2 * self.T * N * K)
         sh = self.shape
         H, I = sh.hidden, sh.inter
@@ -234,7 +246,7 @@ class Workload:
         h = self.ws[off[3]:off[3] + 4 * T * I].view(torch.float32).view(T, I)
         fn = lambda c: tb.bitlinear_gate_up_act(q, s, sq, self.copies[c]["gate"], self.copies[c]["up"], I, self.act,
                                                 out=h)
-        return ("k_gemv_mma<ffn> (gate/up + act)", fn, 2 * tb.i2s_packed_bytes(I, H), 4 * T * I * H)
+        return ("k_gemm_tc<ffn> (gate/up + act)", fn, 2 * tb.i2s_packed_bytes(I, H), 4 * T * I * H)
 
 
 def time_steps(wl: Workload, steps: int, warmup: int, use_graph: bool, e2e: bool):
@@ -433,7 +445,9 @@ def main():
     e2e_val = world * per_step_units * args.steps / (ms_e2e / 1e3)
 
     hbm, bf16, src = peaks()
-    kernel_files = ["ternary_bitlinear_quantized_b200/csrc/gemv.cuh", "ternary_bitlinear_quantized_b200/csrc/common.cuh"]
+    kernel_files = (["ternary_bitlinear_quantized_b200/csrc/engine.cuh"] if decode else
+                    ["ternary_bitlinear_quantized_b200/csrc/gemm_tc.cuh"]) + [
+        "ternary_bitlinear_quantized_b200/csrc/gemv.cuh", "ternary_bitlinear_quantized_b200/csrc/common.cuh"]
     if decode:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,

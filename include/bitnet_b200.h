@@ -136,8 +136,9 @@ size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I);
 
 /* Byte offsets inside that workspace, so that a caller can read the intermediates after
  * a call: off[0] q_x int8 [T,H], off[1] s_x fp32 [T], off[2] sum_x int32 [T],
- * off[3] h fp32 [T,I], off[4] q_h int8 [T,I], off[5] s_h fp32 [T], off[6] sum_h int32 [T].
- * `off` is a HOST array of 7 entries.  Returns BITNET_ERR_SHAPE on invalid sizes. */
+ * off[3] h fp32 [T,I], off[4] q_h int8 [T,I], off[5] s_h fp32 [T], off[6] sum_h int32 [T],
+ * off[7] 256 bytes of grid-barrier counters.  `off` is a HOST array of 8 entries.
+ * Returns BITNET_ERR_SHAPE on invalid sizes. */
 bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size_t* off);
 
 /* The BitNet FFN block on x [T, H]:
@@ -151,13 +152,49 @@ bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size
  * [I2S] "bitnet-b1.58: squared-ReLU FFN" (relu2 vs SiLU from config).
  * p_gate, p_up: I2_S [I, H]; p_down: I2_S [H, I]; H % 128 == 0 and I % 128 == 0.
  * ws: device workspace of at least bitnet_ffn_workspace_bytes(T, H, I) bytes (16-byte
- * aligned).  Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
+ * aligned).  Its barrier counters (off[7]) must be ZERO before the first call (allocate it
+ * zeroed once); every call leaves them zero, except a call that ends in
+ * BITNET_ERR_TIMEOUT, after which they must be zeroed again.  Up to 16 tokens the whole
+ * block is one launch (grid barriers between the dependent steps); more tokens run as
+ * separate launches on the tensor-core path.  Two calls that share a workspace must not
+ * run concurrently.  Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
 bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn,
                                const uint8_t* p_gate, const uint8_t* p_up,
                                const float* g_sub, const uint8_t* p_down,
                                int64_t T, int64_t H, int64_t I, bitnet_act act, float eps,
                                void* out, bitnet_dtype ot, void* ws, size_t ws_bytes,
                                bitnet_stream s);
+
+/* Workspace of bitnet_decoder_block, in bytes (0 if a size is invalid).  NQ = the q (and
+ * o-input) width, usually H. */
+size_t bitnet_block_workspace_bytes(int64_t T, int64_t H, int64_t NQ, int64_t I);
+
+/* Byte offsets inside that workspace: off[0..2] q, s, sum of x (attn_norm) [T,H];
+ * off[3..5] the same for the attention output (attn_sub_norm) [T,NQ]; off[6] the FFN's
+ * workspace (layout of bitnet_ffn_workspace_offsets).  `off`: HOST array of 7 entries. */
+bitnet_status bitnet_block_workspace_offsets(int64_t T, int64_t H, int64_t NQ, int64_t I, size_t* off);
+
+/* The BitLinear projections of one BitNet decoder block, in dependency order:
+ *   q, k, v = BitLinear_{p_q, p_k, p_v}(rmsnorm_quant(x, g_attn_norm))      -> out_q/k/v
+ *   o       = BitLinear_{p_o}(rmsnorm_quant(attn_out, g_attn_sub_norm))       -> out_o [T,H]
+ *   ffn     = bitnet_ffn_block(o; g_ffn_norm, gate, up, g_ffn_sub_norm, down) -> out_ffn [T,H]
+ * x [T,H] and attn_out [T,NQ] are the block input and the attention output (the
+ * attention itself, rotary embedding and residual adds are not part of this call).
+ * Shapes: p_q [NQ,H], p_k / p_v [NKV,H], p_o [H,NQ], p_gate / p_up [I,H], p_down [H,I].
+ * [RMS] BitLinear with BitNetRMSNorm on its input, BitNetMLP.forward with ffn_sub_norm;
+ * [IQ1] the per-block norm weights attn_norm, attn_sub_norm, ffn_norm, ffn_sub_norm.
+ * Outputs are bf16 or fp32 (ot).  Up to 16 tokens the block is ONE launch; the workspace
+ * (bitnet_block_workspace_bytes) follows the rules of bitnet_ffn_block (zero it once).
+ * Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
+bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_dtype xt,
+                                   const float* g_attn_norm, const float* g_attn_sub_norm,
+                                   const float* g_ffn_norm, const float* g_ffn_sub_norm,
+                                   const uint8_t* p_q, const uint8_t* p_k, const uint8_t* p_v,
+                                   const uint8_t* p_o, const uint8_t* p_gate, const uint8_t* p_up,
+                                   const uint8_t* p_down, int64_t T, int64_t H, int64_t NQ,
+                                   int64_t NKV, int64_t I, bitnet_act act, float eps, void* out_q,
+                                   void* out_k, void* out_v, void* out_o, void* out_ffn,
+                                   bitnet_dtype ot, void* ws, size_t ws_bytes, bitnet_stream s);
 
 /* Synchronises `s`, then reads and clears the device status word of the current
  * device: BITNET_OK, or BITNET_ERR_TIMEOUT if a kernel gave up a bounded wait since

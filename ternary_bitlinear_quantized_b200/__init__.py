@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "lib", "i2s_packed_bytes", "pack_i2s", "rmsnorm_quant_act", "bitlinear", "bitlinear_group", "bitlinear_gate_up_act",
-    "ffn_workspace_bytes", "ffn_workspace_offsets", "ffn_block", "device_status", "BitnetError",
+    "ffn_workspace_bytes", "ffn_workspace_offsets", "ffn_block", "block_workspace_bytes", "block_workspace_offsets",
+    "decoder_block", "device_status", "BitnetError",
     "BF16", "F32", "RELU2", "SILU",
 ]
 
@@ -31,7 +32,8 @@ _STATUS = {0: "ok", 1: "null pointer", 2: "invalid shape", 3: "pointer not 16-by
 EXPORTS = [
     "bitnet_i2s_packed_bytes", "bitnet_pack_i2s", "bitnet_rmsnorm_quant_act", "bitnet_bitlinear",
     "bitnet_bitlinear_group", "bitnet_bitlinear_gate_up_act", "bitnet_ffn_workspace_bytes", "bitnet_ffn_workspace_offsets",
-    "bitnet_ffn_block", "bitnet_get_device_status", "bitnet_status_string", "bitnet_last_error",
+    "bitnet_ffn_block", "bitnet_block_workspace_bytes", "bitnet_block_workspace_offsets", "bitnet_decoder_block",
+    "bitnet_get_device_status", "bitnet_status_string", "bitnet_last_error",
 ]
 
 
@@ -67,6 +69,11 @@ def lib() -> ctypes.CDLL:
         "bitnet_ffn_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_p]),
         "bitnet_ffn_block": (c_i, [c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_i,
                                    c_p, c_sz, c_p]),
+        "bitnet_block_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64]),
+        "bitnet_block_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_i64, c_p]),
+        "bitnet_decoder_block": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
+                                       c_i64, c_i64, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_p, c_p, c_p, c_p, c_i,
+                                       c_p, c_sz, c_p]),
         "bitnet_get_device_status": (c_i, [c_p]),
         "bitnet_status_string": (ctypes.c_char_p, [c_i]),
         "bitnet_last_error": (ctypes.c_char_p, []),
@@ -182,7 +189,7 @@ def ffn_workspace_bytes(T: int, H: int, I: int) -> int:
 
 
 def ffn_workspace_offsets(T: int, H: int, I: int) -> list[int]:
-    off = (ctypes.c_size_t * 7)()
+    off = (ctypes.c_size_t * 8)()
     _check(lib().bitnet_ffn_workspace_offsets(T, H, I, ctypes.cast(off, ctypes.c_void_p)), "ffn_workspace_offsets")
     return list(off)
 
@@ -196,11 +203,47 @@ def ffn_block(x, g_ffn, p_gate, p_up, g_sub, p_down, I: int, act: int = RELU2, e
         out = torch.empty(T, H, dtype=out_dtype, device=x.device)
     nws = ffn_workspace_bytes(T, H, I)
     if ws is None:
-        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device)
+        ws = torch.zeros(max(nws, 16), dtype=torch.uint8, device=x.device)  # barrier counters start at zero
     _check(lib().bitnet_ffn_block(_ptr(x), _dtype_code(x.dtype), _ptr(g_ffn), _ptr(p_gate), _ptr(p_up), _ptr(g_sub),
                                   _ptr(p_down), T, H, I, act, eps, _ptr(out), _dtype_code(out.dtype), _ptr(ws),
                                   ws.numel(), _stream(stream)), "ffn_block")
     return out
+
+
+def block_workspace_bytes(T: int, H: int, NQ: int, I: int) -> int:
+    return int(lib().bitnet_block_workspace_bytes(T, H, NQ, I))
+
+
+def block_workspace_offsets(T: int, H: int, NQ: int, I: int) -> list[int]:
+    off = (ctypes.c_size_t * 7)()
+    _check(lib().bitnet_block_workspace_offsets(T, H, NQ, I, ctypes.cast(off, ctypes.c_void_p)),
+           "block_workspace_offsets")
+    return list(off)
+
+
+def decoder_block(x, attn_out, gains: dict, packed: dict, NKV: int, I: int, act: int = RELU2, eps: float = 1e-6,
+                  out_dtype=torch.bfloat16, outs=None, ws=None, stream=None):
+    """The BitLinear projections of a decoder block.  gains: attn_norm, attn_sub_norm,
+    ffn_norm, ffn_sub_norm (tensors or None); packed: q, k, v, o, gate, up, down.
+    Returns dict q, k, v, o, ffn.  ``ws`` must start zeroed (allocated here if None)."""
+    _need(x, "x")
+    _need(attn_out, "attn_out")
+    T, H = x.shape
+    NQ = attn_out.shape[1]
+    if outs is None:
+        e = lambda n: torch.empty(T, n, dtype=out_dtype, device=x.device)
+        outs = {"q": e(NQ), "k": e(NKV), "v": e(NKV), "o": e(H), "ffn": e(H)}
+    if ws is None:
+        ws = torch.zeros(block_workspace_bytes(T, H, NQ, I), dtype=torch.uint8, device=x.device)
+    g = lambda k: _ptr(gains.get(k))
+    _check(lib().bitnet_decoder_block(_ptr(x), _ptr(attn_out), _dtype_code(x.dtype), g("attn_norm"),
+                                      g("attn_sub_norm"), g("ffn_norm"), g("ffn_sub_norm"), _ptr(packed["q"]),
+                                      _ptr(packed["k"]), _ptr(packed["v"]), _ptr(packed["o"]), _ptr(packed["gate"]),
+                                      _ptr(packed["up"]), _ptr(packed["down"]), T, H, NQ, NKV, I, act, eps,
+                                      _ptr(outs["q"]), _ptr(outs["k"]), _ptr(outs["v"]), _ptr(outs["o"]),
+                                      _ptr(outs["ffn"]), _dtype_code(outs["ffn"].dtype), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "decoder_block")
+    return outs
 
 
 def device_status(stream=None) -> int:

@@ -1,6 +1,6 @@
 // The C ABI of include/bitnet_b200.h: argument checks, launch configuration and the
 // order of launches on the caller's stream.  Every step of the arithmetic runs in the
-// kernels of quant.cuh, pack.cuh, gemv.cuh and gemm_tc.cuh (one translation unit, so
+// kernels of quant.cuh, pack.cuh, engine.cuh and gemm_tc.cuh (one translation unit, so
 // that the device status word needs no relocatable device code).
 #include <cstdio>
 #include <cstring>
@@ -10,7 +10,7 @@
 #include "quant.cuh"
 #include "pack.cuh"
 #include "gemv.cuh"
-#include "decode.cuh"
+#include "engine.cuh"
 #include "gemm_tc.cuh"
 
 namespace bitnet {
@@ -200,6 +200,130 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
   return BITNET_OK;
 }
 
+// ------------------------------------------------------------------ decode engine plans
+constexpr int ENG_SLOT_TARGET = 16 * 1024;  // bytes of one ring slot (a stage of 16 rows)
+constexpr int ENG_LOCAL_MAX_TK = 16 * 1024; // T * K up to which every CTA quantises for itself
+
+// K-chunking of one GEMV phase so that a stage (16 rows x chunk, x2 for gate/up) fits a slot.
+static void eng_chunks(EngPhase& p) {
+  const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
+  const int row_bytes = p.K / 4;
+  int max_cb = (ENG_SLOT_TARGET / (GEMV_ROWS * NT) - ENG_ROW_PAD) / 64 * 64;
+  if (max_cb < 64) max_cb = 64;
+  int n = (row_bytes + max_cb - 1) / max_cb;
+  const int cb = ((row_bytes + n - 1) / n + 63) / 64 * 64;
+  n = (row_bytes + cb - 1) / cb;
+  p.chunk_bytes = cb;
+  p.n_chunks = n;
+  p.row_stride = cb + ENG_ROW_PAD;
+  p.stage_bytes = GEMV_ROWS * p.row_stride * NT;
+}
+
+static EngPhase eng_gemv(int K, bool ffn, int n_tensors, const uint8_t* const* packed, const int64_t* N,
+                         void* const* out, int32_t* const* dbg, int out_dtype, int act, float* h) {
+  EngPhase p;
+  memset(&p, 0, sizeof(p));
+  p.kind = ffn ? PH_GEMV_FFN : PH_GEMV;
+  p.K = K;
+  p.n_tensors = n_tensors;
+  int tiles = 0;
+  for (int i = 0; i < n_tensors; ++i) {
+    p.t[i].packed = packed[i];
+    p.t[i].out = out ? out[i] : nullptr;
+    p.t[i].acc_debug = dbg ? dbg[i] : nullptr;
+    p.t[i].N = (int)N[i];
+    p.t[i].tile_begin = tiles;
+    if (!ffn || i == 0) tiles += (int)((N[i] + GEMV_ROWS - 1) / GEMV_ROWS);
+  }
+  p.n_tiles = tiles;
+  p.out_dtype = out_dtype;
+  p.act = act;
+  p.h = h;
+  p.wait_barrier = p.arrive_barrier = -1;
+  eng_chunks(p);
+  return p;
+}
+
+static void eng_src_global(EngPhase& p, const int8_t* q, const float* s, const int32_t* sq) {
+  p.src = SRC_GLOBAL;
+  p.q = const_cast<int8_t*>(q);
+  p.s = const_cast<float*>(s);
+  p.sq = const_cast<int32_t*>(sq);
+}
+
+static void eng_src_local(EngPhase& p, const void* x, int x_f32, const float* gain, int8_t* q_copy, float* s_copy,
+                          int32_t* sq_copy) {
+  p.src = SRC_LOCAL;
+  p.x = x;
+  p.x_f32 = x_f32;
+  p.gain = gain;
+  p.q = q_copy;
+  p.s = s_copy;
+  p.sq = sq_copy;
+}
+
+static EngPhase eng_quant(const void* x, int x_f32, int K, const float* gain, int8_t* q, float* s, int32_t* sq) {
+  EngPhase p;
+  memset(&p, 0, sizeof(p));
+  p.kind = PH_QUANT;
+  p.K = K;
+  p.x = x;
+  p.x_f32 = x_f32;
+  p.gain = gain;
+  p.q = q;
+  p.s = s;
+  p.sq = sq;
+  p.wait_barrier = p.arrive_barrier = -1;
+  return p;
+}
+
+static bool eng_local_ok(int64_t T, int64_t K) { return T * K <= ENG_LOCAL_MAX_TK && K <= ENG_LOCAL_MAX_K; }
+
+// Launch the engine over the phases in `a` (a.T, a.eps, a.n_phases, a.ph, a.counters set).
+static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
+  const int sms = device_sm_count();
+  bool multi = a.n_phases > 1;
+  int max_tiles = 1;
+  for (int i = 0; i < a.n_phases; ++i)
+    if (a.ph[i].kind != PH_QUANT && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
+  const int grid = multi ? sms : (max_tiles < sms ? max_tiles : sms);
+  int acc_ints = 0, qs = 0, slot = 0;
+  for (int i = 0; i < a.n_phases; ++i) {
+    const EngPhase& p = a.ph[i];
+    if (p.kind == PH_QUANT) continue;
+    const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
+    const int per = (p.n_tiles + grid - 1) / grid * NT * 256;
+    if (per > acc_ints) acc_ints = per;
+    if (p.src == SRC_LOCAL && a.T * p.K > qs) qs = a.T * p.K;
+    if (p.stage_bytes > slot) slot = p.stage_bytes;
+  }
+  qs = (qs + 127) / 128 * 128;
+  const int tg = a.T <= 8 ? 1 : 2;
+  void (*kern)(const EngArgs) = tg == 1 ? k_engine<1> : k_engine<2>;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, (const void*)kern);
+  if (e != cudaSuccess) return cuda_fail(e, "k_engine attributes");
+  int dev = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  // With up to 8 tokens, two engine CTAs fit on one SM, so the next launch can stream its
+  // weights while this one finishes; with 9..16 tokens one CTA takes the whole SM.
+  const int budget = (tg == 1 ? per_sm / 2 : per_sm) - 1024 - (int)fa.sharedSizeBytes;
+  int slots = (budget - acc_ints * 4 - qs) / (slot + 16);
+  if (slots > 32) slots = 32;
+  if (slots < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_engine shared memory");
+  a.n_slots = slots;
+  a.slot_bytes = slot;
+  a.acc_ints = acc_ints;
+  a.qs_bytes = qs;
+  const size_t smem = (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs;
+  e = opt_in_smem((const void*)kern, 6 + tg - 1);
+  if (e != cudaSuccess) return cuda_fail(e, "k_engine attribute");
+  e = launch(kern, dim3(grid), dim3(ENG_THREADS), smem, s, true, a);
+  if (e != cudaSuccess) return cuda_fail(e, "k_engine");
+  return BITNET_OK;
+}
+
 static bitnet_status enqueue_gemv(const int8_t* q, const float* s_x, const int32_t* sum_q, int n_tensors,
                                   const uint8_t* const* packed, const int64_t* N, void* const* out,
                                   int32_t* const* acc_debug, int64_t T, int64_t K, bitnet_dtype ot,
@@ -225,18 +349,14 @@ static bitnet_status enqueue_gemv(const int8_t* q, const float* s_x, const int32
     if (!ffn || i == 0) tiles += (int)((N[i] + GEMV_ROWS - 1) / GEMV_ROWS);
   }
   a.n_tiles = tiles;
-  cudaError_t e;
-  if (T <= DEC_MAX_T) {
-    int grid = 0;
-    const DecPlan p = plan_decode(tiles, (int)K, ffn, device_sm_count(), &grid);
-    const int tg = T <= 8 ? 1 : 2;
-    void (*kern)(const GemvArgs, const DecPlan) =
-        ffn ? (tg == 1 ? k_decode<true, 1> : k_decode<true, 2>) : (tg == 1 ? k_decode<false, 1> : k_decode<false, 2>);
-    if ((e = opt_in_smem((const void*)kern, (ffn ? 2 : 0) + tg - 1)) != cudaSuccess)
-      return cuda_fail(e, "k_decode attribute");
-    e = launch(kern, dim3(grid), dim3(DEC_THREADS), (size_t)p.smem_bytes, s, true, a, p);
-    if (e != cudaSuccess) return cuda_fail(e, "k_decode");
-    return BITNET_OK;
+  if (T <= ENG_MAX_T) {
+    EngArgs ea;
+    memset(&ea, 0, sizeof(ea));
+    ea.T = (int)T;
+    ea.n_phases = 1;
+    ea.ph[0] = eng_gemv((int)K, ffn, n_tensors, packed, N, out, acc_debug, ot, act, h);
+    eng_src_global(ea.ph[0], q, s_x, sum_q);
+    return enqueue_engine(ea, s);
   }
   return enqueue_gemm_tc(a, ffn, s);
 }
@@ -352,6 +472,9 @@ bitnet_status bitnet_bitlinear_gate_up_act(const int8_t* q, const float* s_x, co
 
 static size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
+constexpr int FFN_WS_SLOTS = 8;
+constexpr size_t ENG_COUNTER_BYTES = 256;  // ENG_MAX_BARRIERS + 1 counters, padded
+
 bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size_t* off) {
   if (!off) return BITNET_ERR_NULL;
   if (T < 0 || H <= 0 || I <= 0) return BITNET_ERR_SHAPE;
@@ -363,13 +486,89 @@ bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size
   off[4] = o; o = align_up(o + (size_t)T * I);      // q_h
   off[5] = o; o = align_up(o + (size_t)T * 4);      // s_h
   off[6] = o; o = align_up(o + (size_t)T * 4);      // sum_h
+  off[7] = o;                                       // grid-barrier counters
   return BITNET_OK;
 }
 
 size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I) {
-  size_t off[7];
+  size_t off[FFN_WS_SLOTS];
   if (bitnet_ffn_workspace_offsets(T, H, I, off) != BITNET_OK) return 0;
-  return align_up(off[6] + (size_t)T * 4);
+  return off[7] + ENG_COUNTER_BYTES;
+}
+
+// Appends the FFN phases (x [T, H] -> out [T, H]) to an engine plan; `bar` is the next
+// free barrier id, `wait0` a barrier the first phase must wait for (-1: none).
+static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32, const float* g_ffn,
+                     const uint8_t* p_gate, const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T,
+                     int64_t H, int64_t I, int act, void* out, int ot, uint8_t* ws) {
+  size_t off[FFN_WS_SLOTS];
+  bitnet_ffn_workspace_offsets(T, H, I, off);
+  int8_t* q_x = reinterpret_cast<int8_t*>(ws + off[0]);
+  float* s_x = reinterpret_cast<float*>(ws + off[1]);
+  int32_t* sum_x = reinterpret_cast<int32_t*>(ws + off[2]);
+  float* h = reinterpret_cast<float*>(ws + off[3]);
+  int8_t* q_h = reinterpret_cast<int8_t*>(ws + off[4]);
+  float* s_h = reinterpret_cast<float*>(ws + off[5]);
+  int32_t* sum_h = reinterpret_cast<int32_t*>(ws + off[6]);
+  const uint8_t* gu[2] = {p_gate, p_up};
+  const int64_t nI[2] = {I, I};
+  EngPhase gate_up = eng_gemv((int)H, true, 2, gu, nI, nullptr, nullptr, BITNET_F32, act, h);
+  if (eng_local_ok(T, H)) {
+    eng_src_local(gate_up, x, x_f32, g_ffn, q_x, s_x, sum_x);
+    gate_up.wait_barrier = wait0;
+  } else {
+    EngPhase qp = eng_quant(x, x_f32, (int)H, g_ffn, q_x, s_x, sum_x);
+    qp.wait_barrier = wait0;
+    qp.arrive_barrier = bar++;
+    ea.ph[ea.n_phases++] = qp;
+    eng_src_global(gate_up, q_x, s_x, sum_x);
+    gate_up.wait_barrier = qp.arrive_barrier;
+  }
+  gate_up.arrive_barrier = bar++;
+  ea.ph[ea.n_phases++] = gate_up;
+  const int64_t nH[1] = {H};
+  void* o[1] = {out};
+  EngPhase down = eng_gemv((int)I, false, 1, &p_down, nH, o, nullptr, ot, act, nullptr);
+  if (eng_local_ok(T, I)) {
+    eng_src_local(down, h, 1, g_sub, q_h, s_h, sum_h);
+    down.wait_barrier = gate_up.arrive_barrier;
+  } else {
+    EngPhase qp = eng_quant(h, 1, (int)I, g_sub, q_h, s_h, sum_h);
+    qp.wait_barrier = gate_up.arrive_barrier;
+    qp.arrive_barrier = bar++;
+    ea.ph[ea.n_phases++] = qp;
+    eng_src_global(down, q_h, s_h, sum_h);
+    down.wait_barrier = qp.arrive_barrier;
+  }
+  ea.ph[ea.n_phases++] = down;
+}
+
+// The FFN as separate launches (prefill): quant, gate/up + act, quant, down.
+static bitnet_status enqueue_ffn_launches(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
+                                          const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T,
+                                          int64_t H, int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot,
+                                          uint8_t* w, cudaStream_t s) {
+  size_t off[FFN_WS_SLOTS];
+  bitnet_ffn_workspace_offsets(T, H, I, off);
+  int8_t* q_x = reinterpret_cast<int8_t*>(w + off[0]);
+  float* s_x = reinterpret_cast<float*>(w + off[1]);
+  int32_t* sum_x = reinterpret_cast<int32_t*>(w + off[2]);
+  float* h = reinterpret_cast<float*>(w + off[3]);
+  int8_t* q_h = reinterpret_cast<int8_t*>(w + off[4]);
+  float* s_h = reinterpret_cast<float*>(w + off[5]);
+  int32_t* sum_h = reinterpret_cast<int32_t*>(w + off[6]);
+  bitnet_status st = enqueue_quant(x, xt, g_ffn, eps, T, H, q_x, s_x, sum_x, s);
+  if (st != BITNET_OK) return st;
+  const uint8_t* gu[2] = {p_gate, p_up};
+  const int64_t nI[2] = {I, I};
+  st = enqueue_gemv(q_x, s_x, sum_x, 2, gu, nI, nullptr, nullptr, T, H, BITNET_F32, true, act, h, s);
+  if (st != BITNET_OK) return st;
+  st = enqueue_quant(h, BITNET_F32, g_sub, eps, T, I, q_h, s_h, sum_h, s);
+  if (st != BITNET_OK) return st;
+  const uint8_t* pd[1] = {p_down};
+  const int64_t nH[1] = {H};
+  void* o[1] = {out};
+  return enqueue_gemv(q_h, s_h, sum_h, 1, pd, nH, o, nullptr, T, I, ot, false, act, nullptr, s);
 }
 
 bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
@@ -389,29 +588,135 @@ bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ff
       !aligned16(ws) || (g_ffn && !aligned16(g_ffn)) || (g_sub && !aligned16(g_sub)))
     return BITNET_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  size_t off[7];
-  bitnet_ffn_workspace_offsets(T, H, I, off);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  if (T > ENG_MAX_T)
+    return enqueue_ffn_launches(x, xt, g_ffn, p_gate, p_up, g_sub, p_down, T, H, I, act, eps, out, ot, w, s);
+  size_t off[FFN_WS_SLOTS];
+  bitnet_ffn_workspace_offsets(T, H, I, off);
+  EngArgs ea;
+  memset(&ea, 0, sizeof(ea));
+  ea.T = (int)T;
+  ea.eps = eps;
+  ea.counters = reinterpret_cast<unsigned*>(w + off[7]);
+  int bar = 0;
+  plan_ffn(ea, bar, -1, x, xt == BITNET_F32, g_ffn, p_gate, p_up, g_sub, p_down, T, H, I, act, out, ot, w);
+  return enqueue_engine(ea, s);
+}
+
+// ---------------------------------------------------------------- decoder block
+bitnet_status bitnet_block_workspace_offsets(int64_t T, int64_t H, int64_t NQ, int64_t I, size_t* off) {
+  if (!off) return BITNET_ERR_NULL;
+  if (T < 0 || H <= 0 || NQ <= 0 || I <= 0) return BITNET_ERR_SHAPE;
+  size_t o = 0;
+  off[0] = o; o = align_up(o + (size_t)T * H);    // q of x (attn_norm)
+  off[1] = o; o = align_up(o + (size_t)T * 4);
+  off[2] = o; o = align_up(o + (size_t)T * 4);
+  off[3] = o; o = align_up(o + (size_t)T * NQ);   // q of the attention output (attn_sub_norm)
+  off[4] = o; o = align_up(o + (size_t)T * 4);
+  off[5] = o; o = align_up(o + (size_t)T * 4);
+  off[6] = o;                                     // the FFN's workspace
+  return BITNET_OK;
+}
+
+size_t bitnet_block_workspace_bytes(int64_t T, int64_t H, int64_t NQ, int64_t I) {
+  size_t off[7];
+  if (bitnet_block_workspace_offsets(T, H, NQ, I, off) != BITNET_OK) return 0;
+  return off[6] + bitnet_ffn_workspace_bytes(T, H, I);
+}
+
+bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_dtype xt, const float* g_attn_norm,
+                                   const float* g_attn_sub_norm, const float* g_ffn_norm, const float* g_ffn_sub_norm,
+                                   const uint8_t* p_q, const uint8_t* p_k, const uint8_t* p_v, const uint8_t* p_o,
+                                   const uint8_t* p_gate, const uint8_t* p_up, const uint8_t* p_down, int64_t T,
+                                   int64_t H, int64_t NQ, int64_t NKV, int64_t I, bitnet_act act, float eps,
+                                   void* out_q, void* out_k, void* out_v, void* out_o, void* out_ffn, bitnet_dtype ot,
+                                   void* ws, size_t ws_bytes, bitnet_stream stream) {
+  if (xt != BITNET_BF16 && xt != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (act != BITNET_RELU2 && act != BITNET_SILU) return BITNET_ERR_DTYPE;
+  if (T < 0 || T > 0x7FFFFFFFll || H <= 0 || NQ <= 0 || NKV <= 0 || I <= 0 || H % 128 || NQ % 128 || I % 128 ||
+      H > BITNET_MAX_K || NQ > BITNET_MAX_K || I > BITNET_MAX_K || NQ > (1 << 30) || NKV > (1 << 30))
+    return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  const void* need[] = {x, attn_out, p_q, p_k, p_v, p_o, p_gate, p_up, p_down, out_q, out_k, out_v, out_o, out_ffn};
+  for (const void* p : need)
+    if (!p) return BITNET_ERR_NULL;
+  if (!ws) return BITNET_ERR_WORKSPACE;
+  if (ws_bytes < bitnet_block_workspace_bytes(T, H, NQ, I)) return BITNET_ERR_WORKSPACE;
+  for (const void* p : need)
+    if (!aligned16(p)) return BITNET_ERR_ALIGN;
+  const void* gains[] = {g_attn_norm, g_attn_sub_norm, g_ffn_norm, g_ffn_sub_norm};
+  for (const void* p : gains)
+    if (p && !aligned16(p)) return BITNET_ERR_ALIGN;
+  if (!aligned16(ws)) return BITNET_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  size_t off[7];
+  bitnet_block_workspace_offsets(T, H, NQ, I, off);
   int8_t* q_x = reinterpret_cast<int8_t*>(w + off[0]);
   float* s_x = reinterpret_cast<float*>(w + off[1]);
   int32_t* sum_x = reinterpret_cast<int32_t*>(w + off[2]);
-  float* h = reinterpret_cast<float*>(w + off[3]);
-  int8_t* q_h = reinterpret_cast<int8_t*>(w + off[4]);
-  float* s_h = reinterpret_cast<float*>(w + off[5]);
-  int32_t* sum_h = reinterpret_cast<int32_t*>(w + off[6]);
-
-  bitnet_status st = enqueue_quant(x, xt, g_ffn, eps, T, H, q_x, s_x, sum_x, s);
-  if (st != BITNET_OK) return st;
-  const uint8_t* gu[2] = {p_gate, p_up};
-  const int64_t nI[2] = {I, I};
-  st = enqueue_gemv(q_x, s_x, sum_x, 2, gu, nI, nullptr, nullptr, T, H, BITNET_F32, true, act, h, s);
-  if (st != BITNET_OK) return st;
-  st = enqueue_quant(h, BITNET_F32, g_sub, eps, T, I, q_h, s_h, sum_h, s);
-  if (st != BITNET_OK) return st;
-  const uint8_t* pd[1] = {p_down};
+  int8_t* q_a = reinterpret_cast<int8_t*>(w + off[3]);
+  float* s_a = reinterpret_cast<float*>(w + off[4]);
+  int32_t* sum_a = reinterpret_cast<int32_t*>(w + off[5]);
+  uint8_t* wf = w + off[6];
+  const uint8_t* pqkv[3] = {p_q, p_k, p_v};
+  const int64_t nqkv[3] = {NQ, NKV, NKV};
+  void* oqkv[3] = {out_q, out_k, out_v};
   const int64_t nH[1] = {H};
-  void* o[1] = {out};
-  return enqueue_gemv(q_h, s_h, sum_h, 1, pd, nH, o, nullptr, T, I, ot, false, act, nullptr, s);
+  void* oo[1] = {out_o};
+  if (T > ENG_MAX_T) {
+    bitnet_status st = enqueue_quant(x, xt, g_attn_norm, eps, T, H, q_x, s_x, sum_x, s);
+    if (st == BITNET_OK) st = enqueue_gemv(q_x, s_x, sum_x, 3, pqkv, nqkv, oqkv, nullptr, T, H, ot, false, act, nullptr, s);
+    if (st == BITNET_OK) st = enqueue_quant(attn_out, xt, g_attn_sub_norm, eps, T, NQ, q_a, s_a, sum_a, s);
+    if (st == BITNET_OK) st = enqueue_gemv(q_a, s_a, sum_a, 1, &p_o, nH, oo, nullptr, T, NQ, ot, false, act, nullptr, s);
+    if (st == BITNET_OK)
+      st = enqueue_ffn_launches(out_o, ot, g_ffn_norm, p_gate, p_up, g_ffn_sub_norm, p_down, T, H, I, act, eps,
+                                out_ffn, ot, wf, s);
+    return st;
+  }
+  // One engine launch: o first (the FFN depends on it), then q/k/v while o's barrier
+  // completes, then the FFN.
+  size_t offf[FFN_WS_SLOTS];
+  bitnet_ffn_workspace_offsets(T, H, I, offf);
+  EngArgs ea;
+  memset(&ea, 0, sizeof(ea));
+  ea.T = (int)T;
+  ea.eps = eps;
+  ea.counters = reinterpret_cast<unsigned*>(wf + offf[7]);
+  int bar = 0;
+  const int xf = xt == BITNET_F32;
+  EngPhase po = eng_gemv((int)NQ, false, 1, &p_o, nH, oo, nullptr, ot, act, nullptr);
+  EngPhase pqkvp = eng_gemv((int)H, false, 3, pqkv, nqkv, oqkv, nullptr, ot, act, nullptr);
+  int qa_bar = -1, qx_bar = -1;
+  if (!eng_local_ok(T, NQ)) {
+    EngPhase qp = eng_quant(attn_out, xf, (int)NQ, g_attn_sub_norm, q_a, s_a, sum_a);
+    qp.arrive_barrier = qa_bar = bar++;
+    ea.ph[ea.n_phases++] = qp;
+  }
+  if (!eng_local_ok(T, H)) {
+    EngPhase qp = eng_quant(x, xf, (int)H, g_attn_norm, q_x, s_x, sum_x);
+    qp.arrive_barrier = qx_bar = bar++;
+    ea.ph[ea.n_phases++] = qp;
+  }
+  if (qa_bar >= 0) {
+    eng_src_global(po, q_a, s_a, sum_a);
+    po.wait_barrier = qa_bar;
+  } else {
+    eng_src_local(po, attn_out, xf, g_attn_sub_norm, q_a, s_a, sum_a);
+  }
+  po.arrive_barrier = bar++;
+  ea.ph[ea.n_phases++] = po;
+  if (qx_bar >= 0) {
+    eng_src_global(pqkvp, q_x, s_x, sum_x);
+    pqkvp.wait_barrier = qx_bar;
+  } else {
+    eng_src_local(pqkvp, x, xf, g_attn_norm, q_x, s_x, sum_x);
+  }
+  ea.ph[ea.n_phases++] = pqkvp;
+  plan_ffn(ea, bar, po.arrive_barrier, out_o, ot == BITNET_F32, g_ffn_norm, p_gate, p_up, g_ffn_sub_norm, p_down, T,
+           H, I, act, out_ffn, ot, wf);
+  return enqueue_engine(ea, s);
 }
 
 bitnet_status bitnet_get_device_status(bitnet_stream stream) {

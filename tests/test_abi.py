@@ -75,6 +75,9 @@ def test_status_strings(L):
 
 def test_ffn_workspace_layout(L):
     off = tb.ffn_workspace_offsets(3, 256, 384)
-    assert off == sorted(off) and all(o % 256 == 0 for o in off)
+    assert len(off) == 8 and off == sorted(off) and all(o % 256 == 0 for o in off)
     assert off[1] >= 3 * 256 and off[4] - off[3] >= 3 * 384 * 4
-    assert tb.ffn_workspace_bytes(3, 256, 384) >= off[6] + 12
+    assert tb.ffn_workspace_bytes(3, 256, 384) >= off[7] + 36
+    boff = tb.block_workspace_offsets(3, 256, 256, 384)
+    assert len(boff) == 7 and boff == sorted(boff)
+    assert tb.block_workspace_bytes(3, 256, 256, 384) == boff[6] + tb.ffn_workspace_bytes(3, 256, 384)

@@ -143,7 +143,7 @@ def run_ffn(T, H, I, act, seed, out_dtype=torch.bfloat16, x_dtype=torch.bfloat16
     x = d["x"] if x_dtype == torch.bfloat16 else d["x"].float()
     pr = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in ("gate", "up", "down")}
     pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
-    ws = torch.empty(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
     code = tb.RELU2 if act == "relu2" else tb.SILU
     out = tb.ffn_block(x.to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], d["g_ffn_sub_norm"].to(DEV),
                        pg["down"], I, code, 1e-6, out_dtype, ws=ws)
@@ -155,7 +155,8 @@ def run_ffn(T, H, I, act, seed, out_dtype=torch.bfloat16, x_dtype=torch.bfloat16
 
 @pytest.mark.parametrize("act", ["relu2", "silu"])
 @pytest.mark.parametrize("T,H,I", [(1, 256, 384), (3, 640, 1280), (17, 256, 640), (2, 8192, 512), (10, 1152, 2304),
-                                   (64, 512, 768), (130, 384, 1280)])
+                                   (64, 512, 768), (130, 384, 1280), (3, 8192, 512), (1, 256, 16512),
+                                   (16, 2048, 1024)])
 def test_ffn_block_parity(act, T, H, I):
     out, ws, ref, mid, dt = run_ffn(T, H, I, act, seed=T + H)
     off = tb.ffn_workspace_offsets(T, H, I)
@@ -188,3 +189,43 @@ def test_empty_token_batch_is_noop():
     x = torch.empty(0, 256, dtype=torch.bfloat16, device=DEV)
     qq, _, _ = tb.rmsnorm_quant_act(x, None)
     assert qq.shape == (0, 256)
+
+
+# ----------------------------------------------------------------------------- decoder block
+
+def run_block(T, H, NQ, NKV, I, act, seed, out_dtype=torch.bfloat16, calls=1):
+    sh = workloads.BlockShape("blk-test", hidden=H, n_q=NQ, n_kv=NKV, inter=I, act=act)
+    d = workloads.block_inputs(sh, T, seed)
+    pr = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in sh.tensors()}
+    pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
+    gains = {k[2:]: v.to(DEV) for k, v in d.items() if k.startswith("g_")}
+    code = tb.RELU2 if act == "relu2" else tb.SILU
+    ws = torch.zeros(tb.block_workspace_bytes(T, H, NQ, I), dtype=torch.uint8, device=DEV)
+    outs = [tb.decoder_block(d["x"].to(DEV), d["attn_out"].to(DEV), gains, pg, NKV, I, code, 1e-6, out_dtype, ws=ws)
+            for _ in range(calls)]
+    dt = "bf16" if out_dtype == torch.bfloat16 else "f32"
+    ref = O.decoder_block(bf16_to_np(d["x"]), bf16_to_np(d["attn_out"]), {k: v.numpy() for k, v in
+                          {k[2:]: v for k, v in d.items() if k.startswith("g_")}.items()}, pr, sh.tensors(), act,
+                          1e-6, dt)
+    return outs, ref, dt, ws
+
+
+@pytest.mark.parametrize("T,H,NQ,NKV,I,act", [
+    (1, 256, 256, 128, 384, "relu2"),
+    (1, 2560, 2560, 640, 6912, "relu2"),     # the 2B4T shapes at decode
+    (5, 512, 512, 256, 1024, "silu"),
+    (16, 1024, 1024, 256, 2048, "relu2"),    # T * K above the per-CTA quantisation limit
+    (3, 8192, 1024, 128, 640, "silu"),       # large hidden: QUANT phases
+    (40, 384, 384, 128, 640, "relu2"),       # tensor-core path
+])
+def test_decoder_block_parity(T, H, NQ, NKV, I, act):
+    outs, ref, dt, ws = run_block(T, H, NQ, NKV, I, act, seed=T + H, calls=2)
+    for name in ("q", "k", "v", "o", "ffn"):
+        for o in outs:  # the second call reuses the workspace (its barrier counters were reset)
+            got = out_to_np(o[name])
+            assert_close(got, ref[name], dt)
+            assert np.array_equal(got.view(np.uint32), ref[name].view(np.uint32)), name
+    off = tb.block_workspace_offsets(T, H, NQ, I)
+    offf = tb.ffn_workspace_offsets(T, H, I)
+    counters = ws[off[6] + offf[7]: off[6] + offf[7] + 64].cpu().numpy()
+    assert not counters.any()
