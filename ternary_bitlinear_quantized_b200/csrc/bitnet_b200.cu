@@ -201,14 +201,24 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
 }
 
 // ------------------------------------------------------------------ decode engine plans
-constexpr int ENG_SLOT_TARGET = 16 * 1024;  // bytes of one ring slot (a stage of 16 rows)
-constexpr int ENG_LOCAL_MAX_TK = 16 * 1024; // T * K up to which every CTA quantises for itself
+constexpr int ENG_SLOT_MAX = 40 * 1024;       // bytes of one ring slot at most
+constexpr int ENG_LOCAL_MAX_TK = 16 * 1024;   // T * K up to which every CTA quantises for itself
 
-// K-chunking of one GEMV phase so that a stage (16 rows x chunk, x2 for gate/up) fits a slot.
-static void eng_chunks(EngPhase& p) {
+// Stages of one GEMV phase: a whole 16-row tile per tensor (one contiguous copy each) when
+// it fits a slot, else K-chunks of the rows (one copy per row, rows padded by 64 bytes).
+static void eng_chunks(EngPhase& p, int slot_max = ENG_SLOT_MAX) {
   const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
   const int row_bytes = p.K / 4;
-  int max_cb = (ENG_SLOT_TARGET / (GEMV_ROWS * NT) - ENG_ROW_PAD) / 64 * 64;
+  if (NT * GEMV_ROWS * row_bytes <= slot_max) {
+    p.tile_copy = 1;
+    p.chunk_bytes = row_bytes;
+    p.n_chunks = 1;
+    p.row_stride = row_bytes;
+    p.stage_bytes = NT * GEMV_ROWS * row_bytes;
+    return;
+  }
+  p.tile_copy = 0;
+  int max_cb = (slot_max / (GEMV_ROWS * NT) - ENG_ROW_PAD) / 64 * 64;
   if (max_cb < 64) max_cb = 64;
   int n = (row_bytes + max_cb - 1) / max_cb;
   const int cb = ((row_bytes + n - 1) / n + 63) / 64 * 64;
@@ -277,7 +287,8 @@ static EngPhase eng_quant(const void* x, int x_f32, int K, const float* gain, in
   return p;
 }
 
-static bool eng_local_ok(int64_t T, int64_t K) { return T * K <= ENG_LOCAL_MAX_TK && K <= ENG_LOCAL_MAX_K; }
+static bool eng_local_ok(int64_t T, int64_t K) { return T * K <= ENG_LOCAL_MAX_TK && K <= ENG_REG_MAX_K; }
+static bool eng_quant_ok(int64_t K) { return K <= ENG_LOCAL_MAX_K; }
 
 // Launch the engine over the phases in `a` (a.T, a.eps, a.n_phases, a.ph, a.counters set).
 static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
@@ -287,9 +298,10 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   for (int i = 0; i < a.n_phases; ++i)
     if (a.ph[i].kind != PH_QUANT && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
   const int grid = multi ? sms : (max_tiles < sms ? max_tiles : sms);
-  int acc_ints = 0, qs = 0, slot = 0;
+  int acc_ints = 0, qs = 0, slot = 0, xs = 0;
   for (int i = 0; i < a.n_phases; ++i) {
     const EngPhase& p = a.ph[i];
+    if ((p.kind == PH_QUANT || p.src == SRC_LOCAL) && p.K > ENG_REG_MAX_K && p.K > xs) xs = p.K;
     if (p.kind == PH_QUANT) continue;
     const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
     const int per = (p.n_tiles + grid - 1) / grid * NT * 256;
@@ -303,20 +315,30 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, (const void*)kern);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attributes");
-  int dev = 0, per_sm = 0;
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  // With up to 8 tokens, two engine CTAs fit on one SM, so the next launch can stream its
-  // weights while this one finishes; with 9..16 tokens one CTA takes the whole SM.
-  const int budget = (tg == 1 ? per_sm / 2 : per_sm) - 1024 - (int)fa.sharedSizeBytes;
-  int slots = (budget - acc_ints * 4 - qs) / (slot + 16);
+  int max_optin = 0;
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int budget = max_optin - (int)fa.sharedSizeBytes - 256;
+  // Slots: at least four fit, at most ENG_SLOT_MAX bytes each.
+  const int ring = budget - acc_ints * 4 - qs - xs * 4;
+  int slot_max = ring / 4 - 16;
+  if (slot_max > ENG_SLOT_MAX) slot_max = ENG_SLOT_MAX;
+  slot = 0;
+  for (int i = 0; i < a.n_phases; ++i) {
+    if (a.ph[i].kind == PH_QUANT) continue;
+    eng_chunks(a.ph[i], slot_max);
+    if (a.ph[i].stage_bytes > slot) slot = a.ph[i].stage_bytes;
+  }
+  int slots = ring / (slot + 16);
   if (slots > 32) slots = 32;
   if (slots < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_engine shared memory");
   a.n_slots = slots;
   a.slot_bytes = slot;
   a.acc_ints = acc_ints;
   a.qs_bytes = qs;
-  const size_t smem = (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs;
+  a.xs_floats = xs;
+  const size_t smem = (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4;
   e = opt_in_smem((const void*)kern, 6 + tg - 1);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attribute");
   e = launch(kern, dim3(grid), dim3(ENG_THREADS), smem, s, true, a);
@@ -589,7 +611,7 @@ bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ff
     return BITNET_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
-  if (T > ENG_MAX_T)
+  if (T > ENG_MAX_T || !eng_quant_ok(H) || !eng_quant_ok(I))
     return enqueue_ffn_launches(x, xt, g_ffn, p_gate, p_up, g_sub, p_down, T, H, I, act, eps, out, ot, w, s);
   size_t off[FFN_WS_SLOTS];
   bitnet_ffn_workspace_offsets(T, H, I, off);
@@ -665,7 +687,7 @@ bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_d
   void* oqkv[3] = {out_q, out_k, out_v};
   const int64_t nH[1] = {H};
   void* oo[1] = {out_o};
-  if (T > ENG_MAX_T) {
+  if (T > ENG_MAX_T || !eng_quant_ok(H) || !eng_quant_ok(NQ) || !eng_quant_ok(I)) {
     bitnet_status st = enqueue_quant(x, xt, g_attn_norm, eps, T, H, q_x, s_x, sum_x, s);
     if (st == BITNET_OK) st = enqueue_gemv(q_x, s_x, sum_x, 3, pqkv, nqkv, oqkv, nullptr, T, H, ot, false, act, nullptr, s);
     if (st == BITNET_OK) st = enqueue_quant(attn_out, xt, g_attn_sub_norm, eps, T, NQ, q_a, s_a, sum_a, s);

@@ -34,13 +34,13 @@
 
 namespace bitnet {
 
-constexpr int ENG_CONS_WARPS = 8;
+constexpr int ENG_CONS_WARPS = 15;  // + 1 producer warp = 16 warps, 4 per SM sub-partition
 constexpr int ENG_CONS = ENG_CONS_WARPS * 32;
 constexpr int ENG_THREADS = ENG_CONS + 32;
 constexpr int ENG_MAX_PHASES = 8;
 constexpr int ENG_MAX_BARRIERS = 8;
 constexpr int ENG_ROW_PAD = 64;
-constexpr int ENG_LOCAL_MAX_K = 8192;  // local quantisation keeps <= 32 values per thread
+constexpr int ENG_LOCAL_MAX_K = 28672;  // rows staged in shared memory as fp32 (112 KB)
 constexpr int ENG_MAX_T = 16;
 
 enum { PH_GEMV = 0, PH_GEMV_FFN = 1, PH_QUANT = 2 };
@@ -67,33 +67,68 @@ struct EngPhase {
   int out_dtype, act;
   float* h;           // FFN output [T, N] fp32
   int wait_barrier, arrive_barrier;  // -1: none
+  int tile_copy;      // 1: one contiguous bulk copy per tensor and tile; 0: per-row chunks
   int chunk_bytes, n_chunks, row_stride, stage_bytes;
 };
 
-struct EngArgs {
+struct alignas(16) EngArgs {
   int T;
   float eps;
   int n_phases;
   unsigned* counters;  // ENG_MAX_BARRIERS + 1 words in the workspace (last: exit count)
-  int n_slots, slot_bytes, acc_ints, qs_bytes;
+  int n_slots, slot_bytes, acc_ints, qs_bytes, xs_floats;
   EngPhase ph[ENG_MAX_PHASES];
 };
 
 // ------------------------------------------------------------------ consumer-group helpers
 BN_DEV void cons_sync() { named_sync(1, ENG_CONS); }
 
-template <typename T, typename Op>
-BN_DEV T cons_reduce(T v, T* scratch, Op op) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+// Reductions over the 256 consumer threads.  The scratch has two halves used in turn, so
+// one named barrier per reduction suffices: a thread can only overwrite a half after every
+// thread has passed the barrier of the reduction in between, i.e. has read that half.
+struct ConsRed {
+  long long* buf;  // [2][ENG_CONS_WARPS]
+  int flip;
+  BN_DEV long long* next() {
+    long long* b = buf + flip * ENG_CONS_WARPS;
+    flip ^= 1;
+    return b;
+  }
+};
+
+// max over non-negative floats (their bit patterns order like unsigned integers)
+BN_DEV float cons_max_nonneg(float v, ConsRed& r) {
+  unsigned u = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
+  unsigned* b = reinterpret_cast<unsigned*>(r.next());
+  if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = u;
   cons_sync();
-  if (lane == 0) scratch[warp] = v;
-  cons_sync();
-  T r = scratch[0];
+  unsigned m = 0;
 #pragma unroll
-  for (int w = 1; w < ENG_CONS_WARPS; ++w) r = op(r, scratch[w]);
-  return r;
+  for (int i = 0; i < ENG_CONS_WARPS; ++i) m = max(m, b[i]);
+  return __uint_as_float(m);
+}
+
+BN_DEV int cons_sum_i32(int v, ConsRed& r) {
+  int w = __reduce_add_sync(0xffffffffu, v);
+  int* b = reinterpret_cast<int*>(r.next());
+  if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = w;
+  cons_sync();
+  int t = 0;
+#pragma unroll
+  for (int i = 0; i < ENG_CONS_WARPS; ++i) t += b[i];
+  return t;
+}
+
+BN_DEV long long cons_sum_i64(long long v, ConsRed& r) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  long long* b = r.next();
+  if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
+  cons_sync();
+  long long t = 0;
+#pragma unroll
+  for (int w = 0; w < ENG_CONS_WARPS; ++w) t += b[w];
+  return t;
 }
 
 // Load 8 activations (bf16 or fp32) at element offset k of row x, bypassing L1 (the row
@@ -114,68 +149,80 @@ BN_DEV void load8(const void* x, int x_f32, long long k, float* o) {
   }
 }
 
-// RMSNorm + absmax int8 of one row of K <= ENG_LOCAL_MAX_K values held in registers by
-// the 256 consumer threads (thread i owns elements 8(i + 256 j) .. +7).  Writes q (into
-// `qdst`, shared or global), s_x and sum_q (thread 0).  Same operation sequence as
-// quant.cuh: exact fixed-point sum of x^2, fp32 steps without contraction.
-BN_DEV void quant_row_regs(const void* xrow, int x_f32, int K, const float* gain, float eps, int8_t* qdst,
-                           float* s_dst, int32_t* sq_dst, void* red) {
+// RMSNorm + absmax int8 of one row of K <= ENG_REG_MAX_K values by the 256 consumer threads,
+// values in registers (thread i owns elements 8(i + 256 j) .. +7, j < 4).  The activation
+// and gain loads are issued together, so the row costs one memory round trip.  Writes q
+// (into `qdst`, shared or global memory), s_x and sum_q (thread 0).  The same operation
+// sequence as quant.cuh: exact fixed-point sum of x^2 (x^2 and its scaling by 2^e are exact
+// in fp64), fp32 steps without contraction.
+constexpr int ENG_REG_GROUPS = 3;
+constexpr int ENG_REG_MAX_K = 8192;
+static_assert(ENG_CONS * 8 * ENG_REG_GROUPS >= ENG_REG_MAX_K, "register quantiser covers the row");
+
+__device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, const float* gain, float eps,
+                                            int8_t* qdst, float* s_dst, int32_t* sq_dst, long long* red) {
   const int tid = threadIdx.x;
-  float v[4][8];
-  float am = 0.0f;
+  ConsRed R{red, 0};
+  float v[ENG_REG_GROUPS][8], g[ENG_REG_GROUPS][8];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < ENG_REG_GROUPS; ++j) {
     const int k = 8 * (tid + ENG_CONS * j);
     if (k < K) {
       load8(xrow, x_f32, k, v[j]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
+      if (gain != nullptr) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain + k));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain + k + 4));
+        g[j][0] = g0.x; g[j][1] = g0.y; g[j][2] = g0.z; g[j][3] = g0.w;
+        g[j][4] = g1.x; g[j][5] = g1.y; g[j][6] = g1.z; g[j][7] = g1.w;
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[j][i] = 0.0f;
     }
   }
-  am = cons_reduce(am, reinterpret_cast<float*>(red), MaxOp());
+  float am = 0.0f;
+#pragma unroll
+  for (int j = 0; j < ENG_REG_GROUPS; ++j)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
+  am = cons_max_nonneg(am, R);
   float a = am;
   if (gain != nullptr) {
     float ms = 0.0f;
     if (am > 0.0f) {
-      const double M = __dmul_rn((double)am, (double)am);
-      const int e = fixed_point_exponent(M, K);
+      const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
       const double p2e = pow2_f64(e);
       long long part = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < ENG_REG_GROUPS; ++j) {
+        if (8 * (tid + ENG_CONS * j) < K) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const double d = (double)v[j][i];
-          part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
+          for (int i = 0; i < 8; ++i) {
+            const double d = (double)v[j][i];
+            part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
+          }
         }
-      const long long S = cons_reduce(part, reinterpret_cast<long long*>(red), AddOpLL());
-      ms = fixed_point_mean(S, e, K);
+      }
+      ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     float ay = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = 8 * (tid + ENG_CONS * j);
-      if (k < K) {
-        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain + k));
-        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain + k + 4));
-        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    for (int j = 0; j < ENG_REG_GROUPS; ++j) {
+      if (8 * (tid + ENG_CONS * j) < K) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          v[j][i] = __fmul_rn(__fmul_rn(v[j][i], inv), g[i]);
+          v[j][i] = __fmul_rn(__fmul_rn(v[j][i], inv), g[j][i]);
           ay = fmaxf(ay, fabsf(v[j][i]));
         }
       }
     }
-    a = cons_reduce(ay, reinterpret_cast<float*>(red), MaxOp());
+    a = cons_max_nonneg(ay, R);
   }
   const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
   int sum = 0;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < ENG_REG_GROUPS; ++j) {
     const int k = 8 * (tid + ENG_CONS * j);
     if (k < K) {
       uint32_t w[2] = {0u, 0u};
@@ -189,74 +236,91 @@ BN_DEV void quant_row_regs(const void* xrow, int x_f32, int K, const float* gain
       *reinterpret_cast<uint2*>(qdst + k) = make_uint2(w[0], w[1]);
     }
   }
-  sum = cons_reduce(sum, reinterpret_cast<int*>(red), AddOpI());
+  sum = cons_sum_i32(sum, R);
   if (tid == 0) {
     *s_dst = s;
     *sq_dst = sum;
   }
 }
 
-// The same for any K, streaming the row from global memory in four passes (used when a
-// CTA quantises whole tokens for everyone: the QUANT phase).
-BN_DEV void quant_row_stream(const void* xrow, int x_f32, int K, const float* gain, float eps, int8_t* qdst,
-                             float* s_dst, int32_t* sq_dst, void* red) {
+// The same for rows longer than ENG_REG_MAX_K: the row is staged once in shared memory as
+// fp32 (`xs`, K floats) and each pass is a compact rolled loop.
+__device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K, const float* gain, float eps,
+                                              int8_t* qdst, float* s_dst, int32_t* sq_dst, long long* red,
+                                              float* xs) {
   const int tid = threadIdx.x;
-  float v[8];
+  ConsRed R{red, 0};
   float am = 0.0f;
-  for (int k = 8 * tid; k < K; k += 8 * ENG_CONS) {
+  int k = 8 * tid;
+  for (; k + 3 * 8 * ENG_CONS < K; k += 4 * 8 * ENG_CONS) {  // four loads in flight per thread
+    float v[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) load8(xrow, x_f32, k + j * 8 * ENG_CONS, v[j]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      *reinterpret_cast<float4*>(xs + k + j * 8 * ENG_CONS) = make_float4(v[j][0], v[j][1], v[j][2], v[j][3]);
+      *reinterpret_cast<float4*>(xs + k + j * 8 * ENG_CONS + 4) = make_float4(v[j][4], v[j][5], v[j][6], v[j][7]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
+    }
+  }
+  for (; k < K; k += 8 * ENG_CONS) {
+    float v[8];
     load8(xrow, x_f32, k, v);
+    *reinterpret_cast<float4*>(xs + k) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(xs + k + 4) = make_float4(v[4], v[5], v[6], v[7]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
   }
-  am = cons_reduce(am, reinterpret_cast<float*>(red), MaxOp());
-  float a = am, inv = 1.0f;
+  am = cons_max_nonneg(am, R);  // its barrier also orders the xs writes
+  float a = am;
   if (gain != nullptr) {
     float ms = 0.0f;
     if (am > 0.0f) {
-      const double M = __dmul_rn((double)am, (double)am);
-      const int e = fixed_point_exponent(M, K);
+      const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
       const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int k = 8 * tid; k < K; k += 8 * ENG_CONS) {
-        load8(xrow, x_f32, k, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const double d = (double)v[i];
-          part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
-        }
+      for (int kk = tid; kk < K; kk += ENG_CONS) {
+        const double d = (double)xs[kk];
+        part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
       }
-      const long long S = cons_reduce(part, reinterpret_cast<long long*>(red), AddOpLL());
-      ms = fixed_point_mean(S, e, K);
+      ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
     }
-    inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     float ay = 0.0f;
-    for (int k = 8 * tid; k < K; k += 8 * ENG_CONS) {
-      load8(xrow, x_f32, k, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ay = fmaxf(ay, fabsf(__fmul_rn(__fmul_rn(v[i], inv), __ldg(gain + k + i))));
+    for (int kk = tid; kk < K; kk += ENG_CONS) {
+      const float y = __fmul_rn(__fmul_rn(xs[kk], inv), __ldg(gain + kk));
+      xs[kk] = y;
+      ay = fmaxf(ay, fabsf(y));
     }
-    a = cons_reduce(ay, reinterpret_cast<float*>(red), MaxOp());
+    a = cons_max_nonneg(ay, R);  // also orders the xs rewrites
   }
   const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
   int sum = 0;
-  for (int k = 8 * tid; k < K; k += 8 * ENG_CONS) {
-    load8(xrow, x_f32, k, v);
+  for (int kk = 8 * tid; kk < K; kk += 8 * ENG_CONS) {
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float y = gain != nullptr ? __fmul_rn(__fmul_rn(v[i], inv), __ldg(gain + k + i)) : v[i];
-      int qv = __float2int_rn(__fmul_rn(y, s));
+      int qv = __float2int_rn(__fmul_rn(xs[kk + i], s));
       qv = min(127, max(-128, qv));
       sum += qv;
       w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
     }
-    *reinterpret_cast<uint2*>(qdst + k) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint2*>(qdst + kk) = make_uint2(w[0], w[1]);
   }
-  sum = cons_reduce(sum, reinterpret_cast<int*>(red), AddOpI());
+  sum = cons_sum_i32(sum, R);
   if (tid == 0) {
     *s_dst = s;
     *sq_dst = sum;
   }
+}
+
+BN_DEV void quant_row(const void* xrow, int x_f32, int K, const float* gain, float eps, int8_t* qdst, float* s_dst,
+                      int32_t* sq_dst, long long* red, float* xs) {
+  if (K <= ENG_REG_MAX_K)
+    quant_row_regs(xrow, x_f32, K, gain, eps, qdst, s_dst, sq_dst, red);
+  else
+    quant_row_staged(xrow, x_f32, K, gain, eps, qdst, s_dst, sq_dst, red, xs);
 }
 
 // ------------------------------------------------------------------ grid barriers
@@ -291,17 +355,30 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 
 // ------------------------------------------------------------------ the kernel
 template <int TG>
-__global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const EngArgs a) {
+__global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant__ EngArgs args) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // The phase descriptors are read many times with run-time indices; reading them from the
+  // kernel-parameter space costs a constant-cache miss (a memory round trip) on every first
+  // touch of a line, so they are copied to shared memory once, with 16-byte loads.
+  __shared__ EngArgs s_args;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(&args);
+    uint4* dst = reinterpret_cast<uint4*>(&s_args);
+    for (int i = threadIdx.x; i < (int)(sizeof(EngArgs) / 16); i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
+  const EngArgs& a = s_args;
   volatile __shared__ int s_abort;
-  __shared__ long long s_red[ENG_CONS_WARPS];
+  __shared__ __align__(16) long long s_red[2 * ENG_CONS_WARPS];
   __shared__ float s_loc_s[ENG_MAX_T];
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
+  __shared__ float s_beta[ENG_MAX_PHASES][4];
 
   uint8_t* ring = smem;
   const uint32_t bar0 = smem_addr(smem + a.n_slots * a.slot_bytes);
   int* acc = reinterpret_cast<int*>(smem + a.n_slots * a.slot_bytes + 16 * a.n_slots);
   int8_t* qs = reinterpret_cast<int8_t*>(acc + a.acc_ints);
+  float* xs = reinterpret_cast<float*>(qs + a.qs_bytes);  // fp32 staging of one activation row
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (a.n_slots + s); };
 
@@ -315,6 +392,15 @@ __global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const E
     }
     s_abort = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < ENG_MAX_PHASES * 4) {  // per-tensor scales (weights: no dependency wait needed)
+    const int pi = threadIdx.x >> 2, u = threadIdx.x & 3;
+    float b = 0.0f;
+    if (pi < a.n_phases && a.ph[pi].kind != PH_QUANT && u < a.ph[pi].n_tensors) {
+      const EngTensor& t = a.ph[pi].t[u];
+      b = __ldg(reinterpret_cast<const float*>(t.packed + (long long)t.N * (a.ph[pi].K >> 2)));
+    }
+    s_beta[pi][u] = b;
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -356,12 +442,21 @@ __global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const E
           const int cb = min(p.chunk_bytes, row_bytes - c * p.chunk_bytes);
           if (lane == 0) mbar_arrive_expect_tx(full(slot), (uint32_t)(nrows * cb * NT));
           __syncwarp();
-          for (int idx = lane; idx < nrows * NT; idx += 32) {
-            const int u = idx / nrows, r = idx % nrows;
-            const uint8_t* src =
-                p.t[NT == 2 ? u : ti].packed + (long long)(n0 + r) * row_bytes + (long long)c * p.chunk_bytes;
-            bulk_g2s(smem_addr(ring + slot * a.slot_bytes + (u * GEMV_ROWS + r) * p.row_stride), src, (uint32_t)cb,
-                     full(slot));
+          if (p.tile_copy) {
+            // The tile's rows are contiguous: one copy per tensor.
+            if (lane < NT) {
+              const uint8_t* src = p.t[NT == 2 ? lane : ti].packed + (long long)n0 * row_bytes;
+              bulk_g2s(smem_addr(ring + slot * a.slot_bytes + lane * GEMV_ROWS * p.row_stride), src,
+                       (uint32_t)(nrows * row_bytes), full(slot));
+            }
+          } else {
+            for (int idx = lane; idx < nrows * NT; idx += 32) {
+              const int u = idx / nrows, r = idx % nrows;
+              const uint8_t* src =
+                  p.t[NT == 2 ? u : ti].packed + (long long)(n0 + r) * row_bytes + (long long)c * p.chunk_bytes;
+              bulk_g2s(smem_addr(ring + slot * a.slot_bytes + (u * GEMV_ROWS + r) * p.row_stride), src, (uint32_t)cb,
+                       full(slot));
+            }
           }
         }
       }
@@ -386,8 +481,8 @@ __global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const E
       }
       if (p.kind == PH_QUANT) {
         for (int t = blockIdx.x; t < T; t += gridDim.x) {
-          quant_row_stream(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32,
-                           p.K, p.gain, a.eps, p.q + (long long)t * p.K, p.s + t, p.sq + t, s_red);
+          quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
+                    p.gain, a.eps, p.q + (long long)t * p.K, p.s + t, p.sq + t, s_red, xs);
         }
         if (p.arrive_barrier >= 0) grid_arrive(a.counters + p.arrive_barrier);
         continue;
@@ -400,8 +495,8 @@ __global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const E
       const bool local = p.src == SRC_LOCAL;
       if (local) {
         for (int t = 0; t < T; ++t) {
-          quant_row_regs(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32,
-                         p.K, p.gain, a.eps, qs + t * p.K, s_loc_s + t, s_loc_sq + t, s_red);
+          quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
+                    p.gain, a.eps, qs + t * p.K, s_loc_s + t, s_loc_sq + t, s_red, xs);
         }
         if (blockIdx.x == 0 && p.q != nullptr) {  // one copy for callers that read the intermediates
           for (int i = threadIdx.x; i < T * p.K / 16; i += ENG_CONS)
@@ -534,10 +629,10 @@ __global__ void __launch_bounds__(ENG_THREADS, TG == 1 ? 2 : 1) k_engine(const E
         const float sx = local ? s_loc_s[t] : __ldcg(p.s + t);
         const int* at = acc + tl * NT * 256;
         const int accA = at[row * 16 + t] - sq;
-        const float betaA = __ldg(reinterpret_cast<const float*>(p.t[ti].packed + (long long)N * row_bytes));
+        const float betaA = s_beta[pi][ti];
         const float vA = dequant(accA, __fdiv_rn(betaA, sx));
         if (NT == 2) {
-          const float betaU = __ldg(reinterpret_cast<const float*>(p.t[1].packed + (long long)N * row_bytes));
+          const float betaU = s_beta[pi][1];
           const int accU = at[256 + row * 16 + t] - sq;
           const float vU = dequant(accU, __fdiv_rn(betaU, sx));
           p.h[(long long)t * N + n] = ffn_act(vA, vU, p.act);
