@@ -108,6 +108,20 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor of 32-bit words [rows, cols] (row stride `stride` bytes), box box_cols x box_rows.
+static bool make_map_u32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
+                         uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ quant
 static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T, int64_t K,
                                    int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
@@ -204,29 +218,28 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
 constexpr int ENG_SLOT_MAX = 40 * 1024;       // bytes of one ring slot at most
 constexpr int ENG_LOCAL_MAX_TK = 16 * 1024;   // T * K up to which every CTA quantises for itself
 
-// Stages of one GEMV phase: a whole 16-row tile per tensor (one contiguous copy each) when
-// it fits a slot, else K-chunks of the rows (one copy per row, rows padded by 64 bytes).
-static void eng_chunks(EngPhase& p, int slot_max = ENG_SLOT_MAX) {
+// Stage geometry of one GEMV phase: K-chunks of at most 256 32-bit words (the TMA box
+// limit), a multiple of 16 words (one 64-byte consumer step); m_tiles consecutive tiles
+// per stage while the stage fits `slot_max` and does not exceed the tiles a CTA owns.
+static void eng_chunks(EngPhase& p, int slot_max = ENG_SLOT_MAX, int tiles_per_cta = 16) {
   const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-  const int row_bytes = p.K / 4;
-  if (NT * GEMV_ROWS * row_bytes <= slot_max) {
-    p.tile_copy = 1;
-    p.chunk_bytes = row_bytes;
-    p.n_chunks = 1;
-    p.row_stride = row_bytes;
-    p.stage_bytes = NT * GEMV_ROWS * row_bytes;
-    return;
+  const int W = p.K / 16;
+  int n = (W + 255) / 256;
+  int C = ((W + n - 1) / n + 15) / 16 * 16;
+  while (NT * GEMV_ROWS * C * 4 > slot_max && C > 16) {
+    ++n;
+    C = ((W + n - 1) / n + 15) / 16 * 16;
   }
-  p.tile_copy = 0;
-  int max_cb = (slot_max / (GEMV_ROWS * NT) - ENG_ROW_PAD) / 64 * 64;
-  if (max_cb < 64) max_cb = 64;
-  int n = (row_bytes + max_cb - 1) / max_cb;
-  const int cb = ((row_bytes + n - 1) / n + 63) / 64 * 64;
-  n = (row_bytes + cb - 1) / cb;
-  p.chunk_bytes = cb;
+  n = (W + C - 1) / C;
+  int m = slot_max / (NT * GEMV_ROWS * C * 4);
+  if (m > tiles_per_cta) m = tiles_per_cta;
+  if (m > 16) m = 16;
+  if (m < 1) m = 1;
+  p.chunk_words = C;
   p.n_chunks = n;
-  p.row_stride = cb + ENG_ROW_PAD;
-  p.stage_bytes = GEMV_ROWS * p.row_stride * NT;
+  p.m_tiles = m;
+  p.box_rows = GEMV_ROWS * m;
+  p.stage_bytes = NT * p.box_rows * C * 4;
 }
 
 static EngPhase eng_gemv(int K, bool ffn, int n_tensors, const uint8_t* const* packed, const int64_t* N,
@@ -292,6 +305,7 @@ static bool eng_quant_ok(int64_t K) { return K <= ENG_LOCAL_MAX_K; }
 
 // Launch the engine over the phases in `a` (a.T, a.eps, a.n_phases, a.ph, a.counters set).
 static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
+  static_assert(sizeof(EngArgs) % 16 == 0, "EngArgs is copied with 16-byte loads");
   const int sms = device_sm_count();
   bool multi = a.n_phases > 1;
   int max_tiles = 1;
@@ -311,7 +325,7 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   }
   qs = (qs + 127) / 128 * 128;
   const int tg = a.T <= 8 ? 1 : 2;
-  void (*kern)(const EngArgs) = tg == 1 ? k_engine<1> : k_engine<2>;
+  void (*kern)(const EngArgs, const EngMaps) = tg == 1 ? k_engine<1> : k_engine<2>;
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, (const void*)kern);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attributes");
@@ -319,17 +333,25 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   cudaGetDevice(&dev);
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int budget = max_optin - (int)fa.sharedSizeBytes - 256;
+  const int budget = max_optin - (int)fa.sharedSizeBytes - 1024 - 256;  // 1024: ring alignment
   // Slots: at least four fit, at most ENG_SLOT_MAX bytes each.
   const int ring = budget - acc_ints * 4 - qs - xs * 4;
   int slot_max = ring / 4 - 16;
   if (slot_max > ENG_SLOT_MAX) slot_max = ENG_SLOT_MAX;
   slot = 0;
+  EngMaps maps;
+  memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < a.n_phases; ++i) {
-    if (a.ph[i].kind == PH_QUANT) continue;
-    eng_chunks(a.ph[i], slot_max);
-    if (a.ph[i].stage_bytes > slot) slot = a.ph[i].stage_bytes;
+    EngPhase& p = a.ph[i];
+    if (p.kind == PH_QUANT) continue;
+    eng_chunks(p, slot_max, (p.n_tiles + grid - 1) / grid);
+    if (p.stage_bytes > slot) slot = p.stage_bytes;
+    for (int u = 0; u < p.n_tensors; ++u)
+      if (!make_map_u32(&maps.m[i][u], p.t[u].packed, (uint64_t)(p.K / 16), (uint64_t)p.t[u].N, (uint64_t)(p.K / 4),
+                        (uint32_t)p.chunk_words, (uint32_t)p.box_rows))
+        return cuda_fail(cudaErrorInvalidValue, "tensor map (engine weights)");
   }
+  slot = (slot + 127) / 128 * 128;
   int slots = ring / (slot + 16);
   if (slots > 32) slots = 32;
   if (slots < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_engine shared memory");
@@ -338,10 +360,10 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   a.acc_ints = acc_ints;
   a.qs_bytes = qs;
   a.xs_floats = xs;
-  const size_t smem = (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4;
+  const size_t smem = 1024 + (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4;
   e = opt_in_smem((const void*)kern, 6 + tg - 1);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attribute");
-  e = launch(kern, dim3(grid), dim3(ENG_THREADS), smem, s, true, a);
+  e = launch(kern, dim3(grid), dim3(ENG_THREADS), smem, s, true, a, maps);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine");
   return BITNET_OK;
 }

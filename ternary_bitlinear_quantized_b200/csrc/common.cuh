@@ -86,6 +86,14 @@ BN_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar
                : "memory");
 }
 
+// 2-D TMA load of one box of `map` at (x, y) into this CTA's shared memory, completing on
+// barrier `bar` (no multicast).  x * element size must be a multiple of 16 bytes.
+BN_DEV void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
+  asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+               ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
+               : "memory");
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 BN_DEV void named_sync(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 // Named barrier that also returns whether `pred` was true in any of the threads.

@@ -29,6 +29,8 @@
 // first launch; the last CTA to finish zeroes them again.  Every wait is bounded (about
 // a second); a wait that gives up sets BITNET_ERR_TIMEOUT in the device status word.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 #include "gemv.cuh"
 
@@ -39,7 +41,6 @@ constexpr int ENG_CONS = ENG_CONS_WARPS * 32;
 constexpr int ENG_THREADS = ENG_CONS + 32;
 constexpr int ENG_MAX_PHASES = 8;
 constexpr int ENG_MAX_BARRIERS = 8;
-constexpr int ENG_ROW_PAD = 64;
 constexpr int ENG_LOCAL_MAX_K = 28672;  // rows staged in shared memory as fp32 (112 KB)
 constexpr int ENG_MAX_T = 16;
 
@@ -67,8 +68,14 @@ struct EngPhase {
   int out_dtype, act;
   float* h;           // FFN output [T, N] fp32
   int wait_barrier, arrive_barrier;  // -1: none
-  int tile_copy;      // 1: one contiguous bulk copy per tensor and tile; 0: per-row chunks
-  int chunk_bytes, n_chunks, row_stride, stage_bytes;
+  // Stage geometry: a stage is one 2-D TMA box per tensor of box_rows = 16 * m_tiles rows
+  // (m_tiles consecutive 16-row tiles of one tensor) x chunk_words 32-bit words (a K-chunk).
+  int chunk_words, n_chunks, m_tiles, box_rows, stage_bytes;
+};
+
+// One tensor map per tensor and phase: the packed rows viewed as [N, K/16] 32-bit words.
+struct alignas(64) EngMaps {
+  CUtensorMap m[ENG_MAX_PHASES][4];
 };
 
 struct alignas(16) EngArgs {
@@ -355,7 +362,8 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 
 // ------------------------------------------------------------------ the kernel
 template <int TG>
-__global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant__ EngArgs args) {
+__global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant__ EngArgs args,
+                                                            const __grid_constant__ EngMaps maps) {
   extern __shared__ __align__(128) uint8_t smem[];
   // The phase descriptors are read many times with run-time indices; reading them from the
   // kernel-parameter space costs a constant-cache miss (a memory round trip) on every first
@@ -374,9 +382,10 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
   __shared__ float s_beta[ENG_MAX_PHASES][4];
 
-  uint8_t* ring = smem;
-  const uint32_t bar0 = smem_addr(smem + a.n_slots * a.slot_bytes);
-  int* acc = reinterpret_cast<int*>(smem + a.n_slots * a.slot_bytes + 16 * a.n_slots);
+  // TMA boxes land 1024-byte aligned.
+  uint8_t* ring = smem + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
+  const uint32_t bar0 = smem_addr(ring + a.n_slots * a.slot_bytes);
+  int* acc = reinterpret_cast<int*>(ring + a.n_slots * a.slot_bytes + 16 * a.n_slots);
   int8_t* qs = reinterpret_cast<int8_t*>(acc + a.acc_ints);
   float* xs = reinterpret_cast<float*>(qs + a.qs_bytes);  // fp32 staging of one activation row
   auto full = [&](int s) { return bar0 + 8u * s; };
@@ -416,20 +425,28 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     n0 = (tile - p.t[ti].tile_begin) * GEMV_ROWS;
     nrows = min(GEMV_ROWS, p.t[ti].N - n0);
   };
+  // The stage group starting at tile g0: up to m_tiles tiles of the same tensor, ending at
+  // g1; n0 is its first row.
+  auto group = [&](const EngPhase& p, int g0, int te, int& ti, int& n0, int& g1) {
+    int nr;
+    locate(p, g0, ti, n0, nr);
+    const int tensor_end = (p.kind == PH_GEMV && ti + 1 < p.n_tensors) ? p.t[ti + 1].tile_begin : p.n_tiles;
+    g1 = min(min(te, tensor_end), g0 + p.m_tiles);
+  };
 
   if (warp == ENG_CONS_WARPS) {
     // ------------------------------------------------------------ producer
+    // One elected lane per tensor issues a 2-D TMA box per stage (no multicast).
     int st = 0;
     for (int pi = 0; pi < a.n_phases && !s_abort; ++pi) {
       const EngPhase& p = a.ph[pi];
       if (p.kind == PH_QUANT) continue;
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-      const int row_bytes = p.K >> 2;
       int tb, te;
       tile_range(p, tb, te);
-      for (int tile = tb; tile < te && !s_abort; ++tile) {
-        int ti, n0, nrows;
-        locate(p, tile, ti, n0, nrows);
+      for (int g0 = tb; g0 < te && !s_abort;) {
+        int ti, n0, g1;
+        group(p, g0, te, ti, n0, g1);
         for (int c = 0; c < p.n_chunks; ++c, ++st) {
           const int slot = st % a.n_slots;
           bool ok = true;
@@ -439,26 +456,13 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
             s_abort = 1;
             break;
           }
-          const int cb = min(p.chunk_bytes, row_bytes - c * p.chunk_bytes);
-          if (lane == 0) mbar_arrive_expect_tx(full(slot), (uint32_t)(nrows * cb * NT));
+          if (lane == 0) mbar_arrive_expect_tx(full(slot), (uint32_t)p.stage_bytes);
           __syncwarp();
-          if (p.tile_copy) {
-            // The tile's rows are contiguous: one copy per tensor.
-            if (lane < NT) {
-              const uint8_t* src = p.t[NT == 2 ? lane : ti].packed + (long long)n0 * row_bytes;
-              bulk_g2s(smem_addr(ring + slot * a.slot_bytes + lane * GEMV_ROWS * p.row_stride), src,
-                       (uint32_t)(nrows * row_bytes), full(slot));
-            }
-          } else {
-            for (int idx = lane; idx < nrows * NT; idx += 32) {
-              const int u = idx / nrows, r = idx % nrows;
-              const uint8_t* src =
-                  p.t[NT == 2 ? u : ti].packed + (long long)(n0 + r) * row_bytes + (long long)c * p.chunk_bytes;
-              bulk_g2s(smem_addr(ring + slot * a.slot_bytes + (u * GEMV_ROWS + r) * p.row_stride), src, (uint32_t)cb,
-                       full(slot));
-            }
-          }
+          if (lane < NT)
+            tma_load_2d(smem_addr(ring + slot * a.slot_bytes + lane * p.box_rows * p.chunk_words * 4),
+                            &maps.m[pi][NT == 2 ? lane : ti], c * p.chunk_words, n0, full(slot));
         }
+        g0 = g1;
       }
     }
   } else {
@@ -521,23 +525,32 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
           for (int g = 0; g < 4; ++g)
 #pragma unroll
             for (int i = 0; i < 4; ++i) f[u][tg][g][i] = 0;
-      bool have = false;
       int gstep = 0;
-      for (int tile = tb; tile < te && !s_abort; ++tile) {
-        int ti, n0, nrows;
-        locate(p, tile, ti, n0, nrows);
+      const int W = p.K >> 4;  // 32-bit words per row
+      for (int g0 = tb; g0 < te && !s_abort;) {
+        int ti, n0, g1;
+        group(p, g0, te, ti, n0, g1);
+        const int N = p.t[ti].N;
         for (int c = 0; c < p.n_chunks; ++c, ++st) {
           const int slot = st % a.n_slots;
-          const int cb = min(p.chunk_bytes, row_bytes - c * p.chunk_bytes);
+          const int cb = 4 * min(p.chunk_words, W - c * p.chunk_words);  // bytes of this chunk per row
           const int nsteps = (cb + 63) >> 6;
-          const int first = (warp - gstep % ENG_CONS_WARPS + ENG_CONS_WARPS) % ENG_CONS_WARPS;
+          const int pitch = 4 * p.chunk_words;                          // row pitch of the box
+          const uint8_t* sbase = ring + slot * a.slot_bytes;
+          bool waited = false;
           if (s_abort) break;
-          if (first < nsteps) {
-            if (!mbar_wait_bounded(full(slot), (st / a.n_slots) & 1)) {
-              s_abort = 1;
-              break;
+          for (int j = 0; j < g1 - g0; ++j) {
+            const int first = (warp - gstep % ENG_CONS_WARPS + ENG_CONS_WARPS) % ENG_CONS_WARPS;
+            gstep += nsteps;
+            if (first >= nsteps) continue;
+            if (!waited) {
+              if (!mbar_wait_bounded(full(slot), (st / a.n_slots) & 1)) {
+                s_abort = 1;
+                break;
+              }
+              waited = true;
             }
-            const uint8_t* sbase = ring + slot * a.slot_bytes;
+            const int nrows = min(GEMV_ROWS, N - n0 - GEMV_ROWS * j);
             for (int step = first; step < nsteps; step += ENG_CONS_WARPS) {
               const int boff = 64 * step + 16 * r;
               const bool valid = boff < cb;
@@ -545,14 +558,14 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
                 if (u < NT) {
-                  const uint8_t* rb = sbase + u * GEMV_ROWS * p.row_stride + boff;
-                  wa[u] = (valid && gid < nrows) ? *reinterpret_cast<const uint4*>(rb + gid * p.row_stride)
+                  const uint8_t* rb = sbase + (u * p.box_rows + GEMV_ROWS * j) * pitch + boff;
+                  wa[u] = (valid && gid < nrows) ? *reinterpret_cast<const uint4*>(rb + gid * pitch)
                                                  : make_uint4(0, 0, 0, 0);
-                  wb[u] = (valid && gid + 8 < nrows) ? *reinterpret_cast<const uint4*>(rb + (gid + 8) * p.row_stride)
+                  wb[u] = (valid && gid + 8 < nrows) ? *reinterpret_cast<const uint4*>(rb + (gid + 8) * pitch)
                                                      : make_uint4(0, 0, 0, 0);
                 }
               }
-              const int kb = 4 * (c * p.chunk_bytes + 64 * step) + 128 * (r >> 1) + 16 * (r & 1);
+              const int kb = 4 * (c * 4 * p.chunk_words + 64 * step) + 128 * (r >> 1) + 16 * (r & 1);
               uint4 xa[4], xb[4];
 #pragma unroll
               for (int g = 0; g < 4; ++g) {
@@ -586,33 +599,28 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
                 }
               }
             }
-            have = true;
-          }
-          gstep += nsteps;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(empty(slot));
-          if (c == p.n_chunks - 1) {
-            if (have) {
-              int* at = acc + (tile - tb) * NT * 256;
+            // This warp's part of tile g0 + j in this stage -> the tile's shared accumulator.
+            int* at = acc + (g0 + j - tb) * NT * 256;
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                if (u < NT) {
+            for (int u = 0; u < 2; ++u) {
+              if (u < NT) {
 #pragma unroll
-                  for (int tg = 0; tg < TG; ++tg)
+                for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                      const int v = (f[u][tg][0][i] >> 6) + (f[u][tg][1][i] >> 4) + (f[u][tg][2][i] >> 2) + f[u][tg][3][i];
-                      const int row = gid + ((i & 2) ? 8 : 0), tok = tg * 8 + 2 * r + (i & 1);
-                      if (tok < T && row < nrows) atomicAdd(at + u * 256 + row * 16 + tok, v);
+                  for (int i = 0; i < 4; ++i) {
+                    const int v = (f[u][tg][0][i] >> 6) + (f[u][tg][1][i] >> 4) + (f[u][tg][2][i] >> 2) + f[u][tg][3][i];
+                    const int row = gid + ((i & 2) ? 8 : 0), tok = tg * 8 + 2 * r + (i & 1);
+                    if (tok < T && row < nrows) atomicAdd(at + u * 256 + row * 16 + tok, v);
 #pragma unroll
-                      for (int g = 0; g < 4; ++g) f[u][tg][g][i] = 0;
-                    }
-                }
+                    for (int g = 0; g < 4; ++g) f[u][tg][g][i] = 0;
+                  }
               }
             }
-            have = false;
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty(slot));
         }
+        g0 = g1;
       }
       if (named_sync_or(1, ENG_CONS, s_abort != 0)) break;
       // Epilogue of this phase's tiles.
