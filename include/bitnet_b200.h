@@ -165,6 +165,29 @@ bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ff
                                void* out, bitnet_dtype ot, void* ws, size_t ws_bytes,
                                bitnet_stream s);
 
+/* The same FFN block for callers that cannot allocate device memory themselves -- for
+ * example a plugin running inside a host framework that owns all device memory and forbids
+ * allocation while it serves, or a process under a hard memory cap.  (The BitNet pages
+ * have no counterpart: this is an interface convenience, not part of the method.)
+ *   - The workspace is a file-scope device array of bitnet_ffn_block_noalloc_max_bytes()
+ *     bytes (4 MiB) inside the library; every GPU that loads the library holds it until
+ *     the process exits.  Sizes whose workspace (bitnet_ffn_workspace_bytes) exceeds it
+ *     are rejected with BITNET_ERR_WORKSPACE (bitnet_last_error() says why).
+ *   - The call allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *     The first call on a device looks up the array's device address on that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call clears the grid-barrier counters of the array with cudaMemsetAsync on `s`
+ *     before it launches; the rest of the array keeps the previous call's contents.
+ *   - All calls share the one array per device, so calls that overlap on the GPU (other
+ *     streams, other threads) race: serialise them.
+ * Arguments, arithmetic and other errors as bitnet_ffn_block (without ws / ws_bytes). */
+size_t bitnet_ffn_block_noalloc_max_bytes(void);
+bitnet_status bitnet_ffn_block_noalloc(const void* x, bitnet_dtype xt, const float* g_ffn,
+                                       const uint8_t* p_gate, const uint8_t* p_up,
+                                       const float* g_sub, const uint8_t* p_down, int64_t T,
+                                       int64_t H, int64_t I, bitnet_act act, float eps, void* out,
+                                       bitnet_dtype ot, bitnet_stream s);
+
 /* Workspace of bitnet_decoder_block, in bytes (0 if a size is invalid).  NQ = the q (and
  * o-input) width, usually H. */
 size_t bitnet_block_workspace_bytes(int64_t T, int64_t H, int64_t NQ, int64_t I);

@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "lib", "i2s_packed_bytes", "pack_i2s", "rmsnorm_quant_act", "bitlinear", "bitlinear_group", "bitlinear_gate_up_act",
-    "ffn_workspace_bytes", "ffn_workspace_offsets", "ffn_block", "block_workspace_bytes", "block_workspace_offsets",
+    "ffn_workspace_bytes", "ffn_workspace_offsets", "ffn_block", "ffn_block_noalloc", "block_workspace_bytes", "block_workspace_offsets",
     "decoder_block", "device_status", "BitnetError",
     "BF16", "F32", "RELU2", "SILU",
 ]
@@ -32,7 +32,8 @@ _STATUS = {0: "ok", 1: "null pointer", 2: "invalid shape", 3: "pointer not 16-by
 EXPORTS = [
     "bitnet_i2s_packed_bytes", "bitnet_pack_i2s", "bitnet_rmsnorm_quant_act", "bitnet_bitlinear",
     "bitnet_bitlinear_group", "bitnet_bitlinear_gate_up_act", "bitnet_ffn_workspace_bytes", "bitnet_ffn_workspace_offsets",
-    "bitnet_ffn_block", "bitnet_block_workspace_bytes", "bitnet_block_workspace_offsets", "bitnet_decoder_block",
+    "bitnet_ffn_block", "bitnet_ffn_block_noalloc_max_bytes", "bitnet_ffn_block_noalloc",
+    "bitnet_block_workspace_bytes", "bitnet_block_workspace_offsets", "bitnet_decoder_block",
     "bitnet_get_device_status", "bitnet_status_string", "bitnet_last_error",
 ]
 
@@ -69,6 +70,9 @@ def lib() -> ctypes.CDLL:
         "bitnet_ffn_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_p]),
         "bitnet_ffn_block": (c_i, [c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_i,
                                    c_p, c_sz, c_p]),
+        "bitnet_ffn_block_noalloc_max_bytes": (c_sz, []),
+        "bitnet_ffn_block_noalloc": (c_i, [c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_i,
+                                           c_p]),
         "bitnet_block_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64]),
         "bitnet_block_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_i64, c_p]),
         "bitnet_decoder_block": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
@@ -207,6 +211,21 @@ def ffn_block(x, g_ffn, p_gate, p_up, g_sub, p_down, I: int, act: int = RELU2, e
     _check(lib().bitnet_ffn_block(_ptr(x), _dtype_code(x.dtype), _ptr(g_ffn), _ptr(p_gate), _ptr(p_up), _ptr(g_sub),
                                   _ptr(p_down), T, H, I, act, eps, _ptr(out), _dtype_code(out.dtype), _ptr(ws),
                                   ws.numel(), _stream(stream)), "ffn_block")
+    return out
+
+
+def ffn_block_noalloc(x, g_ffn, p_gate, p_up, g_sub, p_down, I: int, act: int = RELU2, eps: float = 1e-6,
+                      out_dtype=torch.bfloat16, out=None, stream=None):
+    """ffn_block for callers that cannot allocate device memory: the workspace is the
+    library's built-in device array (shared by all calls on a device; overlapping calls
+    race).  ``out`` must be given by such callers; it is allocated here only for tests."""
+    _need(x, "x")
+    T, H = x.shape
+    if out is None:
+        out = torch.empty(T, H, dtype=out_dtype, device=x.device)
+    _check(lib().bitnet_ffn_block_noalloc(_ptr(x), _dtype_code(x.dtype), _ptr(g_ffn), _ptr(p_gate), _ptr(p_up),
+                                          _ptr(g_sub), _ptr(p_down), T, H, I, act, eps, _ptr(out),
+                                          _dtype_code(out.dtype), _stream(stream)), "ffn_block_noalloc")
     return out
 
 

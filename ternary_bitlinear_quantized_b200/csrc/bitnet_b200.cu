@@ -4,6 +4,7 @@
 // that the device status word needs no relocatable device code).
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -645,6 +646,64 @@ bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ff
   int bar = 0;
   plan_ffn(ea, bar, -1, x, xt == BITNET_F32, g_ffn, p_gate, p_up, g_sub, p_down, T, H, I, act, out, ot, w);
   return enqueue_engine(ea, s);
+}
+
+// ---------------------------------------------------------------- FFN without a caller workspace
+// For callers that cannot allocate device memory themselves (for example a plugin inside a
+// host framework that owns all device memory and forbids allocation while it serves, or a
+// process under a hard memory cap): the FFN block's workspace lives in this file-scope
+// array instead.  Every GPU that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB: every FFN up to 16 tokens of the
+                                                    // configured model shapes fits
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device.  The array's name in host
+// code is only a host-side stand-in, so the address is looked up once per device, with
+// that device current, by the first call made on it.
+static bitnet_status noalloc_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return cuda_fail(cudaErrorInvalidDevice, "no-alloc scratch (device id)");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    addr[dev] = reinterpret_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return BITNET_OK;
+}
+
+size_t bitnet_ffn_block_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
+bitnet_status bitnet_ffn_block_noalloc(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
+                                       const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T,
+                                       int64_t H, int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot,
+                                       bitnet_stream stream) {
+  if (T < 0 || H <= 0 || I <= 0) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  const size_t need = bitnet_ffn_workspace_bytes(T, H, I);
+  if (need == 0) return BITNET_ERR_SHAPE;
+  if (need > kNoAllocScratchBytes) {
+    t_last_error = "bitnet_ffn_block_noalloc: the workspace for these sizes exceeds the built-in scratch of " +
+                   std::to_string(kNoAllocScratchBytes) + " bytes; pass a workspace to bitnet_ffn_block";
+    return BITNET_ERR_WORKSPACE;
+  }
+  uint8_t* ws = nullptr;
+  bitnet_status st = noalloc_scratch(&ws);
+  if (st != BITNET_OK) return st;
+  // The grid-barrier counters must start at zero; the previous call normally leaves them
+  // zero, but clear them anyway (a call that timed out would not have).
+  size_t off[FFN_WS_SLOTS];
+  bitnet_ffn_workspace_offsets(T, H, I, off);
+  cudaError_t e = cudaMemsetAsync(ws + off[7], 0, ENG_COUNTER_BYTES, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
+  return bitnet_ffn_block(x, xt, g_ffn, p_gate, p_up, g_sub, p_down, T, H, I, act, eps, out, ot, ws,
+                          kNoAllocScratchBytes, stream);
 }
 
 // ---------------------------------------------------------------- decoder block
