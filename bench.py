@@ -134,6 +134,46 @@ def stored_traffic(kernel_key: str, sha: str):
     return None
 
 
+def workload_units(name: str):
+    """(packed bytes per step, int8 ops per step, tensor shapes) of a workload, from its shapes."""
+    spec = workloads.WORKLOADS[name]
+    if spec["kind"] == "bitlinear":
+        tensors = {"w": (spec["N"], spec["K"])}
+    else:
+        sh = spec["shape"]
+        names = ["gate", "up", "down"] if spec["kind"] == "ffn" else list(sh.tensors())
+        tensors = {nm: sh.tensors()[nm] for nm in names}
+    T = spec["T"]
+    packed = sum(n * k // 4 + 32 for (n, k) in tensors.values())
+    ops = sum(2 * T * n * k for (n, k) in tensors.values())
+    return packed, ops, tensors
+
+
+def workload_config(name: str, world: int, use_graph: bool) -> dict:
+    """The `config` object of the JSON line (identical for both arms)."""
+    packed, ops, _ = workload_units(name)
+    n_copies = max(1, math.ceil(2 * L2_BYTES / packed) + 1)
+    return {"workload": name, "T": workloads.WORKLOADS[name]["T"], "packed_bytes_per_step": packed,
+            "int8_ops_per_step": ops, "parallelism": f"replicas x{world}",
+            "l2": f"weights rotated over {n_copies} copies ({n_copies * packed / 1e6:.0f} MB > 2x L2)",
+            "cuda_graphs": use_graph}
+
+
+def max_over_ranks(values):
+    """Element-wise maximum of per-rank timings over all ranks (identity with one process)."""
+    t = torch.tensor(values, dtype=torch.float64)
+    if torch.distributed.is_initialized():
+        if torch.distributed.get_backend() == "nccl":
+            t = t.cuda()
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(units_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, over the slowest rank's time."""
+    return world * units_per_step * steps / (ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- workload on the GPU
 
 class Workload:
@@ -407,7 +447,7 @@ def main():
         line = {"metric": metric, "value": val, "unit": u, "n_gpus": args.gpus, "steps": args.steps,
                 "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "impl": "reference", "dtype": "int8", "data": "synthetic",
-                "config": {"workload": args.workload, "T": spec["T"]},
+                "config": workload_config(args.workload, args.gpus, not args.no_graph),
                 "cpu_baseline": {"value": val, "unit": u, "cores": cores, "kind": "oracle", "sample": sample},
                 "e2e": {"value": val, "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -436,13 +476,10 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status}")
 
-    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e])
     per_step_units = wl.packed_bytes / 1e9 if decode else wl.ops_per_step / 1e12
-    value = world * per_step_units * args.steps / (ms / 1e3)
-    e2e_val = world * per_step_units * args.steps / (ms_e2e / 1e3)
+    value = whole_job_rate(per_step_units, args.steps, world, ms)
+    e2e_val = whole_job_rate(per_step_units, args.steps, world, ms_e2e)
 
     hbm, bf16, src = peaks()
     kernel_files = (["ternary_bitlinear_quantized_b200/csrc/engine.cuh"] if decode else
@@ -472,11 +509,7 @@ def main():
             "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": args.workload, "T": wl.T, "packed_bytes_per_step": wl.packed_bytes,
-                       "int8_ops_per_step": wl.ops_per_step, "parallelism": f"replicas x{world}",
-                       "l2": f"weights rotated over {wl.n_copies} copies "
-                             f"({wl.n_copies * wl.packed_bytes / 1e6:.0f} MB > 2x L2)",
-                       "cuda_graphs": use_graph},
+            "config": workload_config(args.workload, world, use_graph),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
