@@ -127,6 +127,25 @@ static bool make_map_u32(CUtensorMap* m, const void* base, uint64_t cols, uint64
 static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T, int64_t K,
                                    int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
   if (T == 0) return BITNET_OK;
+  // Rows of up to 8192 values (K a multiple of 8, 16-byte aligned rows): values in registers.
+  const size_t esz_r = xt == BITNET_BF16 ? 2 : 4;
+  if (K <= 4 * 8 * QR_THREADS && K % 8 == 0 && aligned16(x) && aligned16(q) && (K * esz_r) % 16 == 0) {
+    const int ng = K <= 2048 ? 1 : (K <= 4096 ? 2 : 4);
+    cudaError_t e;
+    if (xt == BITNET_BF16) {
+      auto* kern = ng == 1 ? k_rmsnorm_quant_regs<__nv_bfloat16, 1>
+                           : (ng == 2 ? k_rmsnorm_quant_regs<__nv_bfloat16, 2> : k_rmsnorm_quant_regs<__nv_bfloat16, 4>);
+      e = launch(kern, dim3((unsigned)T), dim3(QR_THREADS), 0, s, true, reinterpret_cast<const __nv_bfloat16*>(x), gain,
+                 eps, (int)K, q, s_x, sum_q);
+    } else {
+      auto* kern = ng == 1 ? k_rmsnorm_quant_regs<float, 1>
+                           : (ng == 2 ? k_rmsnorm_quant_regs<float, 2> : k_rmsnorm_quant_regs<float, 4>);
+      e = launch(kern, dim3((unsigned)T), dim3(QR_THREADS), 0, s, true, reinterpret_cast<const float*>(x), gain, eps,
+                 (int)K, q, s_x, sum_q);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "k_rmsnorm_quant_regs");
+    return BITNET_OK;
+  }
   int threads = (int)((K / 8 + 31) / 32 * 32);
   threads = threads < 128 ? 128 : (threads > 1024 ? 1024 : threads);
   const size_t smem = (size_t)K * sizeof(float);
@@ -168,9 +187,32 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
   a.sum_q = g.sum_q;
   a.T = g.T;
   a.K = g.K;
-  int bn = (g.T + 15) / 16 * 16;
-  const int bn_max = ffn ? 128 : 256;
-  a.BN = bn > bn_max ? bn_max : bn;
+  // Token-tile width: the candidate that minimises waves x (BN + per-tile overhead), so
+  // that the last wave of 128-row tiles is not left nearly empty.
+  {
+    int m_tiles = 0;
+    for (int i = 0; i < g.n_tensors; ++i)
+      if (!ffn || i == 0) m_tiles += (g.t[i].N + TC_BM - 1) / TC_BM;
+    const int sms_ = device_sm_count();
+    const int bn_max = ffn ? 128 : 256;
+    const int cands[4] = {256, 192, 128, 64};
+    long best = -1;
+    int best_bn = 64;
+    for (int c : cands) {
+      int bn = c;
+      const int tfit = (g.T + 15) / 16 * 16;
+      if (bn > bn_max) continue;
+      if (bn > tfit) bn = tfit;
+      const long tiles = (long)m_tiles * ((g.T + bn - 1) / bn);
+      const long waves = (tiles + sms_ - 1) / sms_;
+      const long cost = waves * (bn + 48);
+      if (best < 0 || cost < best) {
+        best = cost;
+        best_bn = bn;
+      }
+    }
+    a.BN = best_bn;
+  }
   a.n_tensors = g.n_tensors;
   a.out_dtype = g.out_dtype;
   a.act = g.act;

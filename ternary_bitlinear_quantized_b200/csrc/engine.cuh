@@ -575,11 +575,13 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
                   xb[g] = (TG > 1 && valid && t_b < T) ? *reinterpret_cast<const uint4*>(qs + t_b * p.K + kb + 32 * g)
                                                        : z;
                 } else {
-                  xa[g] = (valid && t_a < T)
-                              ? __ldcg(reinterpret_cast<const uint4*>(p.q + (long long)t_a * p.K + kb + 32 * g))
-                              : z;
+                  // Plain (L1-cached) loads: this SM has not read these lines before in this
+                  // launch (L1 starts empty), and they were complete when the phase's grid
+                  // barrier was passed.
+                  xa[g] = (valid && t_a < T) ? *reinterpret_cast<const uint4*>(p.q + (long long)t_a * p.K + kb + 32 * g)
+                                             : z;
                   xb[g] = (TG > 1 && valid && t_b < T)
-                              ? __ldcg(reinterpret_cast<const uint4*>(p.q + (long long)t_b * p.K + kb + 32 * g))
+                              ? *reinterpret_cast<const uint4*>(p.q + (long long)t_b * p.K + kb + 32 * g)
                               : z;
                 }
               }

@@ -10,8 +10,8 @@
 //   warp 4      TMA producer: per k-block, the BN x 128 int8 activation tile
 //               (128-byte swizzle, the UMMA K-major canonical layout) and the 128 x 32
 //               byte packed weight tile of each tensor;
-//   warps 6-9   expanders: thread r turns row r's 32 packed bytes into 128 u8 codes and
-//               writes them in the same swizzled K-major layout: field g of packed words
+//   warps 6-13  expanders: two threads per row turn the row's 32 packed bytes into 128 u8
+//               codes and write them in the same swizzled K-major layout: field g of packed words
 //               4h..4h+3 is exactly the 16-byte chunk 2g + h (in-features 32g + 16h ..
 //               +15), placed at chunk position (2g + h) ^ (r % 8);
 //   warp 5      MMA issuer: allocates TMEM, issues 4 MMAs (K = 32 each) per k-block and
@@ -34,11 +34,12 @@ namespace bitnet {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 128;
-constexpr int TC_THREADS = 320;
+constexpr int TC_EXP_WARPS = 8;     // warps 6-13: two threads per tile row
+constexpr int TC_THREADS = (6 + TC_EXP_WARPS) * 32;
 constexpr int TC_EPI_WARPS = 4;      // warps 0-3
 constexpr int TC_TMA_WARP = 4;
 constexpr int TC_MMA_WARP = 5;
-constexpr int TC_EXP_WARP0 = 6;      // warps 6-9
+constexpr int TC_EXP_WARP0 = 6;
 constexpr int TC_MAX_STAGES = 6;
 
 struct TcTensor {
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_tma(s), 1);
-      mbar_init(full_a(s), 128);
+      mbar_init(full_a(s), TC_EXP_WARPS * 32);
       mbar_init(empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -198,7 +199,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     }
   } else if (warp >= TC_EXP_WARP0) {
     // ------------------------------------------------------------ expanders
-    const int r = threadIdx.x - TC_EXP_WARP0 * 32;  // row of the tile
+    // Thread e: row r = e % 128 of the tile, fields 2h and 2h + 1 (h = e / 128), i.e. the
+    // 16-byte chunks 4h .. 4h + 3 of the row's 128 u8 codes.
+    const int e = threadIdx.x - TC_EXP_WARP0 * 32;
+    const int r = e & 127, h = e >> 7;
     int it = 0;
     for (int lin = blockIdx.x; lin < total && !s_abort; lin += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -215,7 +219,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
           asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w1.x), "=r"(w1.y), "=r"(w1.z), "=r"(w1.w) : "r"(pa + 16));
           const uint32_t rowa = sA(s, u) + r * 128;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
+          for (int gg = 0; gg < 2; ++gg) {
+            const int g = 2 * h + gg;
             const int sh = 6 - 2 * g;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {

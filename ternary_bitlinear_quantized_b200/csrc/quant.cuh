@@ -153,4 +153,116 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
   quantise_staged_row(xs, K, gain, eps, q + t * K, s_x + t, sum_q + t, vec != 0, red, amax);
 }
 
+// The same arithmetic for rows of K <= 2048 * NG values held in registers by 256 threads
+// (thread i owns elements 8(i + 256 j) .. +7, j < NG), so a CTA reads its row once and
+// several tokens fit on one SM.  Reductions use one barrier each (two scratch halves used
+// in turn).
+constexpr int QR_THREADS = 256;
+constexpr int QR_WARPS = QR_THREADS / 32;
+
+template <typename T>
+BN_DEV T qr_reduce(T v, T* scratch, int& flip, bool is_max) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const T w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? (v > w ? v : w) : v + w;
+  }
+  T* b = scratch + flip * QR_WARPS;
+  flip ^= 1;
+  if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
+  __syncthreads();
+  T r = b[0];
+#pragma unroll
+  for (int w = 1; w < QR_WARPS; ++w) r = is_max ? (r > b[w] ? r : b[w]) : r + b[w];
+  return r;
+}
+
+template <typename TIn, int NG>
+__global__ void __launch_bounds__(QR_THREADS) k_rmsnorm_quant_regs(const TIn* __restrict__ x,
+                                                                  const float* __restrict__ gain, float eps, int K,
+                                                                  int8_t* __restrict__ q, float* __restrict__ s_x,
+                                                                  int32_t* __restrict__ sum_q) {
+  __shared__ float redf[2 * QR_WARPS];
+  __shared__ long long redl[2 * QR_WARPS];
+  __shared__ int redi[2 * QR_WARPS];
+  int ff = 0, fl = 0, fi = 0;
+  const long long t = blockIdx.x;
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  const TIn* xr = x + t * K;
+  float v[NG][8];
+  float am = 0.0f;
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const int k = 8 * (tid + QR_THREADS * j);
+    if (k < K) {
+      RowLoader<TIn>::load(xr + k, v[j]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[j][i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
+  }
+  am = qr_reduce(am, redf, ff, true);
+  float a = am;
+  if (gain != nullptr) {
+    float ms = 0.0f;
+    if (am > 0.0f) {
+      const double M = __dmul_rn((double)am, (double)am);
+      const int e = fixed_point_exponent(M, K);
+      const double p2e = pow2_f64(e);
+      long long part = 0;
+#pragma unroll
+      for (int j = 0; j < NG; ++j)
+        if (8 * (tid + QR_THREADS * j) < K) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const double d = (double)v[j][i];
+            part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
+          }
+        }
+      ms = fixed_point_mean(qr_reduce(part, redl, fl, false), e, K);
+    }
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    float ay = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      const int k = 8 * (tid + QR_THREADS * j);
+      if (k < K) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[j][i] = __fmul_rn(__fmul_rn(v[j][i], inv), __ldg(gain + k + i));
+          ay = fmaxf(ay, fabsf(v[j][i]));
+        }
+      }
+    }
+    a = qr_reduce(ay, redf, ff, true);
+  }
+  const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+  int sum = 0;
+  int8_t* qr = q + t * K;
+#pragma unroll
+  for (int j = 0; j < NG; ++j) {
+    const int k = 8 * (tid + QR_THREADS * j);
+    if (k < K) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int qv = __float2int_rn(__fmul_rn(v[j][i], s));
+        qv = min(127, max(-128, qv));
+        sum += qv;
+        w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2*>(qr + k) = make_uint2(w[0], w[1]);
+    }
+  }
+  sum = qr_reduce(sum, redi, fi, false);
+  if (tid == 0) {
+    s_x[t] = s;
+    sum_q[t] = sum;
+  }
+}
+
 }  // namespace bitnet
