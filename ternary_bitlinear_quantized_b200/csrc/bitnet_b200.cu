@@ -260,29 +260,28 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
 // ------------------------------------------------------------------ decode engine plans
 constexpr int ENG_SLOT_MAX = 40 * 1024;       // bytes of one ring slot at most
 constexpr int ENG_LOCAL_MAX_TK = 16 * 1024;   // T * K up to which every CTA quantises for itself
+constexpr int ENG_QS_GLOBAL_MAX = 32 * 1024;  // given activations up to this size are staged in shared memory
 
-// Stage geometry of one GEMV phase: K-chunks of at most 256 32-bit words (the TMA box
-// limit), a multiple of 16 words (one 64-byte consumer step); m_tiles consecutive tiles
-// per stage while the stage fits `slot_max` and does not exceed the tiles a CTA owns.
-static void eng_chunks(EngPhase& p, int slot_max = ENG_SLOT_MAX, int tiles_per_cta = 16) {
+// Stage geometry of one GEMV phase: K-chunks of C 32-bit words with C = 16 (mod 32) (a
+// consumer step is 16 words, and the rows of a 16-row box are then 64 (mod 128) bytes apart,
+// so two adjacent rows fall in different halves of the shared-memory banks), C <= 240 (the
+// TMA box limit is 256 elements), and the stage (tensors x 16 rows x C words) within
+// slot_max bytes.  The last chunk of a row may be partly outside the tensor (zero-filled).
+static void eng_chunks(EngPhase& p, int slot_max) {
   const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
   const int W = p.K / 16;
-  int n = (W + 255) / 256;
-  int C = ((W + n - 1) / n + 15) / 16 * 16;
-  while (NT * GEMV_ROWS * C * 4 > slot_max && C > 16) {
-    ++n;
-    C = ((W + n - 1) / n + 15) / 16 * 16;
+  int C = 16;
+  for (int n = 1; n <= W; ++n) {
+    int c = (W + n - 1) / n;
+    c = c <= 16 ? 16 : (c - 16 + 31) / 32 * 32 + 16;
+    if (c <= 240 && NT * 64 * c <= slot_max) {
+      C = c;
+      break;
+    }
   }
-  n = (W + C - 1) / C;
-  int m = slot_max / (NT * GEMV_ROWS * C * 4);
-  if (m > tiles_per_cta) m = tiles_per_cta;
-  if (m > 16) m = 16;
-  if (m < 1) m = 1;
   p.chunk_words = C;
-  p.n_chunks = n;
-  p.m_tiles = m;
-  p.box_rows = GEMV_ROWS * m;
-  p.stage_bytes = NT * p.box_rows * C * 4;
+  p.n_chunks = (W + C - 1) / C;
+  p.stage_bytes = NT * 64 * C;
 }
 
 static EngPhase eng_gemv(int K, bool ffn, int n_tensors, const uint8_t* const* packed, const int64_t* N,
@@ -306,7 +305,6 @@ static EngPhase eng_gemv(int K, bool ffn, int n_tensors, const uint8_t* const* p
   p.act = act;
   p.h = h;
   p.wait_barrier = p.arrive_barrier = -1;
-  eng_chunks(p);
   return p;
 }
 
@@ -355,18 +353,20 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   for (int i = 0; i < a.n_phases; ++i)
     if (a.ph[i].kind != PH_QUANT && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
   const int grid = multi ? sms : (max_tiles < sms ? max_tiles : sms);
-  int acc_ints = 0, qs = 0, slot = 0, xs = 0;
+  int acc_ints = 0, qs = 0, xs = 0;
   for (int i = 0; i < a.n_phases; ++i) {
     const EngPhase& p = a.ph[i];
     if ((p.kind == PH_QUANT || p.src == SRC_LOCAL) && p.K > ENG_REG_MAX_K && p.K > xs) xs = p.K;
     if (p.kind == PH_QUANT) continue;
     const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-    const int per = (p.n_tiles + grid - 1) / grid * NT * 256;
+    const int per = (p.n_tiles + grid - 1) / grid * NT * GEMV_ROWS * a.T;
     if (per > acc_ints) acc_ints = per;
-    if (p.src == SRC_LOCAL && a.T * p.K > qs) qs = a.T * p.K;
-    if (p.stage_bytes > slot) slot = p.stage_bytes;
+    // Activations staged in shared memory: always for SRC_LOCAL, else when they fit.
+    const int xp = (p.K + 255) / 256 * 256 + 64;
+    if ((p.src == SRC_LOCAL || a.T * xp <= ENG_QS_GLOBAL_MAX) && a.T * xp > qs) qs = a.T * xp;
   }
   qs = (qs + 127) / 128 * 128;
+  acc_ints = (acc_ints + 3) / 4 * 4;
   const int tg = a.T <= 8 ? 1 : 2;
   void (*kern)(const EngArgs, const EngMaps) = tg == 1 ? k_engine<1> : k_engine<2>;
   cudaFuncAttributes fa;
@@ -377,26 +377,27 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int budget = max_optin - (int)fa.sharedSizeBytes - 1024 - 256;  // 1024: ring alignment
-  // Slots: at least four fit, at most ENG_SLOT_MAX bytes each.
+  // Slots: about six fit, at most ENG_SLOT_MAX bytes each (larger TMA boxes stream faster
+  // than more, smaller ones).
   const int ring = budget - acc_ints * 4 - qs - xs * 4;
-  int slot_max = ring / 4 - 16;
+  int slot_max = ring / 6 - 16;
   if (slot_max > ENG_SLOT_MAX) slot_max = ENG_SLOT_MAX;
-  slot = 0;
+  int slot = 0;
   EngMaps maps;
   memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < a.n_phases; ++i) {
     EngPhase& p = a.ph[i];
     if (p.kind == PH_QUANT) continue;
-    eng_chunks(p, slot_max, (p.n_tiles + grid - 1) / grid);
+    eng_chunks(p, slot_max);
     if (p.stage_bytes > slot) slot = p.stage_bytes;
     for (int u = 0; u < p.n_tensors; ++u)
       if (!make_map_u32(&maps.m[i][u], p.t[u].packed, (uint64_t)(p.K / 16), (uint64_t)p.t[u].N, (uint64_t)(p.K / 4),
-                        (uint32_t)p.chunk_words, (uint32_t)p.box_rows))
+                        (uint32_t)p.chunk_words, (uint32_t)GEMV_ROWS))
         return cuda_fail(cudaErrorInvalidValue, "tensor map (engine weights)");
   }
   slot = (slot + 127) / 128 * 128;
   int slots = ring / (slot + 16);
-  if (slots > 32) slots = 32;
+  if (slots > ENG_MAX_SLOTS) slots = ENG_MAX_SLOTS;
   if (slots < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_engine shared memory");
   a.n_slots = slots;
   a.slot_bytes = slot;

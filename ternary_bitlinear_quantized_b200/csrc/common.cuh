@@ -35,6 +35,21 @@ BN_DEV uint4 ldg_nc_v4(const void* p) {
   return v;
 }
 
+// 16-byte shared-memory load at a shared-space address.
+BN_DEV uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+// The same, only where `pred` holds; elsewhere `v` keeps its value.
+BN_DEV void lds128_if(uint4& v, uint32_t addr, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "@p ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "r"(addr), "r"((uint32_t)pred));
+}
+
 // ---------------------------------------------------------------- mbarriers, bulk copies
 BN_DEV uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -50,6 +65,9 @@ BN_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 BN_DEV void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+BN_DEV void mbar_arrive_count(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 BN_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;

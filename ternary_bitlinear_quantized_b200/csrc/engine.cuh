@@ -14,11 +14,11 @@
 // is being completed) fills the wait.
 //
 // Weights do not depend on any phase, so a producer warp streams the packed bytes of
-// ALL phases of this CTA, in phase order, through a ring of shared-memory slots with
-// cp.async.bulk; it starts before griddepcontrol.wait, i.e. while the previous kernel
-// on the stream is still running.  Consumer warps (8) work through the stages exactly
-// as in the single-phase decode product (gemv.cuh: one AND per 2-bit field, mma.sync
-// m16n8k32 u8 x s8, per-field accumulators combined exactly).
+// ALL phases of this CTA, in phase order, through a ring of shared-memory slots with 2-D
+// TMA boxes; it starts before griddepcontrol.wait, i.e. while the previous kernel on the
+// stream is still running.  The 15 consumer warps work in groups, each group owning a
+// 16-row tile over all of its K-chunks (one AND per 2-bit field, mma.sync m16n8k32
+// u8 x s8, per-field accumulators combined exactly once per tile).
 //
 // Arithmetic and sources as in quant.cuh ("Add optional RMSNorm support to BitNet
 // quantization": BitNetRMSNorm before quantisation) and gemv.cuh ("fix: I2_S ARM kernel
@@ -43,6 +43,7 @@ constexpr int ENG_MAX_PHASES = 8;
 constexpr int ENG_MAX_BARRIERS = 8;
 constexpr int ENG_LOCAL_MAX_K = 28672;  // rows staged in shared memory as fp32 (112 KB)
 constexpr int ENG_MAX_T = 16;
+constexpr int ENG_MAX_SLOTS = 32;  // ring slots at most
 
 enum { PH_GEMV = 0, PH_GEMV_FFN = 1, PH_QUANT = 2 };
 enum { SRC_GLOBAL = 0, SRC_LOCAL = 1 };
@@ -68,9 +69,10 @@ struct EngPhase {
   int out_dtype, act;
   float* h;           // FFN output [T, N] fp32
   int wait_barrier, arrive_barrier;  // -1: none
-  // Stage geometry: a stage is one 2-D TMA box per tensor of box_rows = 16 * m_tiles rows
-  // (m_tiles consecutive 16-row tiles of one tensor) x chunk_words 32-bit words (a K-chunk).
-  int chunk_words, n_chunks, m_tiles, box_rows, stage_bytes;
+  // Stage geometry: a stage is one 2-D TMA box per tensor of 16 rows (one tile) x
+  // chunk_words 32-bit words (a K-chunk; chunk_words = 16 mod 32, so the rows of a box are
+  // 64 mod 128 bytes apart); stage_bytes = tensors x 64 x chunk_words.
+  int chunk_words, n_chunks, stage_bytes;
 };
 
 // One tensor map per tensor and phase: the packed rows viewed as [N, K/16] 32-bit words.
@@ -156,6 +158,18 @@ BN_DEV void load8(const void* x, int x_f32, long long k, float* o) {
   }
 }
 
+// Activation layout in shared memory.  A consumer lane r (of the four lanes that share a
+// weight row in an m16n8k32 fragment) multiplies, for weight field g of 64-byte step s, the
+// 16 activations k = 256 s + 128 (r >> 1) + 32 g + 16 (r & 1) + j, j < 16.  Storing those 16
+// bytes at 256 s + 64 g + 16 r puts the four lanes' pieces of one field side by side, so a
+// 16-byte load by every lane is served without bank conflicts.  Token rows are
+// round_up(K, 256) + 64 bytes apart (also conflict-free for consecutive tokens).
+BN_DEV int eng_perm(int k) {  // k a multiple of 8
+  const int o = k & 255;
+  return (k & ~255) + 64 * ((o >> 5) & 3) + 32 * (o >> 7) + 16 * ((o >> 4) & 1) + (o & 15);
+}
+BN_DEV int eng_x_pitch(int K) { return ((K + 255) & ~255) + 64; }
+
 // RMSNorm + absmax int8 of one row of K <= ENG_REG_MAX_K values by the 256 consumer threads,
 // values in registers (thread i owns elements 8(i + 256 j) .. +7, j < 4).  The activation
 // and gain loads are issued together, so the row costs one memory round trip.  Writes q
@@ -167,7 +181,7 @@ constexpr int ENG_REG_MAX_K = 8192;
 static_assert(ENG_CONS * 8 * ENG_REG_GROUPS >= ENG_REG_MAX_K, "register quantiser covers the row");
 
 __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, const float* gain, float eps,
-                                            int8_t* qdst, float* s_dst, int32_t* sq_dst, long long* red) {
+                                            int8_t* qdst, bool perm, float* s_dst, int32_t* sq_dst, long long* red) {
   const int tid = threadIdx.x;
   ConsRed R{red, 0};
   float v[ENG_REG_GROUPS][8], g[ENG_REG_GROUPS][8];
@@ -240,7 +254,7 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
         sum += qv;
         w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
       }
-      *reinterpret_cast<uint2*>(qdst + k) = make_uint2(w[0], w[1]);
+      *reinterpret_cast<uint2*>(qdst + (perm ? eng_perm(k) : k)) = make_uint2(w[0], w[1]);
     }
   }
   sum = cons_sum_i32(sum, R);
@@ -253,7 +267,7 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
 // The same for rows longer than ENG_REG_MAX_K: the row is staged once in shared memory as
 // fp32 (`xs`, K floats) and each pass is a compact rolled loop.
 __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K, const float* gain, float eps,
-                                              int8_t* qdst, float* s_dst, int32_t* sq_dst, long long* red,
+                                              int8_t* qdst, bool perm, float* s_dst, int32_t* sq_dst, long long* red,
                                               float* xs) {
   const int tid = threadIdx.x;
   ConsRed R{red, 0};
@@ -313,7 +327,7 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
       sum += qv;
       w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
     }
-    *reinterpret_cast<uint2*>(qdst + kk) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint2*>(qdst + (perm ? eng_perm(kk) : kk)) = make_uint2(w[0], w[1]);
   }
   sum = cons_sum_i32(sum, R);
   if (tid == 0) {
@@ -322,12 +336,13 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
   }
 }
 
-BN_DEV void quant_row(const void* xrow, int x_f32, int K, const float* gain, float eps, int8_t* qdst, float* s_dst,
-                      int32_t* sq_dst, long long* red, float* xs) {
+// `perm`: write q in the shared-memory layout of eng_perm (else plain order).
+BN_DEV void quant_row(const void* xrow, int x_f32, int K, const float* gain, float eps, int8_t* qdst, bool perm,
+                      float* s_dst, int32_t* sq_dst, long long* red, float* xs) {
   if (K <= ENG_REG_MAX_K)
-    quant_row_regs(xrow, x_f32, K, gain, eps, qdst, s_dst, sq_dst, red);
+    quant_row_regs(xrow, x_f32, K, gain, eps, qdst, perm, s_dst, sq_dst, red);
   else
-    quant_row_staged(xrow, x_f32, K, gain, eps, qdst, s_dst, sq_dst, red, xs);
+    quant_row_staged(xrow, x_f32, K, gain, eps, qdst, perm, s_dst, sq_dst, red, xs);
 }
 
 // ------------------------------------------------------------------ grid barriers
@@ -360,6 +375,253 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
   return ok;
 }
 
+// ------------------------------------------------------------------ stage schedule
+// A GEMV phase gives each CTA the tiles [tb, tb + nt) (16 weight rows; the tensors of a
+// group phase concatenated; for the FFN a tile is the gate and the up tile of the same
+// rows).  A stage is one tile x one K-chunk: one 2-D TMA box per tensor.  The consumer
+// warps form ng groups of ENG_CONS_WARPS / ng warps.  A group owns a tile for all of its
+// chunks, so its warps keep their partial sums in registers across the chunks and add
+// them to the tile's shared accumulator once.  Tiles are dealt to the groups in rounds of
+// ng; the tiles of a last, partial round are split by chunks between the groups.
+// Producer and consumers walk the same sequence with this iterator.
+BN_DEV int eng_groups(int nt) { return nt >= 5 ? 5 : (nt >= 3 ? 3 : 1); }
+
+struct EngSched {
+  int nch, ng, R, s, units, maxlen;
+  int a, b, q;
+  bool rem;
+  BN_DEV EngSched(int nt, int nch_) : nch(nch_), a(0), b(0), q(0), rem(false) {
+    ng = eng_groups(nt);
+    R = nt / ng;
+    const int left = nt - R * ng;
+    s = left == 0 ? 1 : (nch >= 2 ? min(ng / left, nch) : 1);
+    units = left * s;
+    maxlen = (nch + s - 1) / s;
+  }
+  // Next stage: owning group, tile (local index), chunk, and whether it is the last chunk
+  // of the group's share of the tile.  False at the end.
+  BN_DEV bool next(int& grp, int& tile, int& c, bool& last) {
+    while (true) {
+      if (!rem) {
+        if (a >= R) {
+          rem = true;
+          a = 0;
+          q = 0;
+          continue;
+        }
+        grp = q;
+        tile = a * ng + q;
+        c = b;
+        last = b == nch - 1;
+        if (++q == ng) {
+          q = 0;
+          if (++b == nch) {
+            b = 0;
+            ++a;
+          }
+        }
+        return true;
+      }
+      if (a >= maxlen || units == 0) return false;
+      const int u = q, i = a;
+      if (++q == units) {
+        q = 0;
+        ++a;
+      }
+      const int k = u % s, cb = nch * k / s, ce = nch * (k + 1) / s;
+      if (cb + i < ce) {
+        grp = u;
+        tile = R * ng + u / s;
+        c = cb + i;
+        last = c == ce - 1;
+        return true;
+      }
+    }
+  }
+};
+
+// Wait until the producer has tagged ring slot `tag` with stage `want` (bounded, like the
+// barrier waits).
+BN_DEV bool wait_slot_tag(const volatile int* tag, int want) {
+  if (*tag == want) return true;
+  const long long t0 = clock64();
+  while (*tag != want) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicExch(&g_device_status, (int)BITNET_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ products of one phase
+// The consumer warp's part of one GEMV phase: walk the stage sequence (advancing the ring
+// position `slot`/`par` for every stage), and for the stages of its group wait for the
+// data, run its share of the 64-byte steps, release the slot, and after the last chunk of
+// a unit add its partial sums to the tile's shared accumulator acc[tile][u][row][token].
+// Lane (gid, r) holds rows gid and gid + 8 of the tile, bytes 16 r .. 16 r + 15 of each
+// step (the A fragments of mma.sync m16n8k32, one AND per 2-bit field), and the
+// activations of tokens gid (and 8 + gid), or of token T - 1 where those do not exist.
+// XSM: activations in shared memory (layout eng_perm, lane addresses xs_a / xs_b); else in
+// global memory in plain order (xg_a / xg_b).  Returns false if a wait gave up.
+template <int TG, int NT, bool XSM>
+__device__ __forceinline__ bool eng_phase_products(const EngArgs& a, const EngPhase& p, int nt, uint32_t ring_s,
+                                                   uint32_t bar0, const volatile int* slot_tag, int& seq,
+                                                   int& slot, uint32_t& par, int* acc, uint32_t xs_a,
+                                                   uint32_t xs_b, const int8_t* xg_a, const int8_t* xg_b) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, r = lane & 3;
+  const int T = a.T;
+  const int ng = eng_groups(nt), gw = ENG_CONS_WARPS / ng;
+  const int my_grp = warp / gw, my_i = warp - my_grp * gw;
+  const int C = p.chunk_words, W = p.K >> 4, pitch = 4 * C;
+  int f[NT][TG][4][4];
+#pragma unroll
+  for (int u = 0; u < NT; ++u)
+#pragma unroll
+    for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[u][tg][g][i] = 0;
+  // This group's stages, in sequence order: in the full rounds every ng-th stage (tile
+  // r * ng + my_grp, chunks 0 .. nch-1); in the last round unit my_grp, whose stage i sits
+  // at i * units + my_grp while every unit still has a chunk i (i < lmin), else after the
+  // units that do.  `pos` is the sequence index of the stage, `done` how far the ring
+  // position (slot, par) has been advanced.
+  const EngSched sc(nt, p.n_chunks);
+  const int nch = p.n_chunks;
+  int rot = 0, done = 0, rr = 0, cc = 0;
+  const int own_full = sc.R * nch;
+  int own_rem = 0, ucb = 0, lmin = 0, rank = 0;
+  if (my_grp < sc.units) {
+    const int k = my_grp % sc.s;
+    ucb = nch * k / sc.s;
+    own_rem = nch * (k + 1) / sc.s - ucb;
+    lmin = nch / sc.s;
+    for (int u = 0; u < my_grp; ++u) {
+      const int ku = u % sc.s;
+      if (nch * (ku + 1) / sc.s - nch * ku / sc.s > lmin) ++rank;
+    }
+  }
+  int rem_len_total = 0;  // stages of the last round
+  for (int u = 0; u < sc.units; ++u) {
+    const int ku = u % sc.s;
+    rem_len_total += nch * (ku + 1) / sc.s - nch * ku / sc.s;
+  }
+  for (int j = 0; j < own_full + own_rem; ++j) {
+    int pos, tl, c;
+    bool last;
+    if (j < own_full) {
+      c = cc;
+      tl = rr * ng + my_grp;
+      pos = (rr * nch + cc) * ng + my_grp;
+      last = cc == nch - 1;
+      if (++cc == nch) {
+        cc = 0;
+        ++rr;
+      }
+    } else {
+      const int i = j - own_full;
+      c = ucb + i;
+      tl = sc.R * ng + my_grp / sc.s;
+      pos = sc.R * ng * nch + (i < lmin ? i * sc.units + my_grp : lmin * sc.units + rank);
+      last = i == own_rem - 1;
+    }
+    // advance the ring position to stage `pos`
+    slot += pos - done;
+    done = pos + 1;
+    while (slot >= a.n_slots) {
+      slot -= a.n_slots;
+      par ^= 1u;
+    }
+    const int s = slot;
+    const uint32_t ph = par;
+    if (++slot == a.n_slots) {
+      slot = 0;
+      par ^= 1u;
+    }
+    // Groups run ahead of one another, so the slot's previous fill may still be in flight;
+    // a parity wait is only unambiguous once the producer has taken the slot for this stage.
+    if (!wait_slot_tag(slot_tag + s, seq + pos)) return false;
+    if (!mbar_wait_bounded(bar0 + 8u * s, ph)) return false;
+    const int cbytes = 4 * min(C, W - c * C);  // bytes of the rows inside the tensor
+    const int nsteps = (cbytes + 63) >> 6;
+    int t = my_i - rot;  // the group's warps take the steps in turn, starting one later each stage
+    if (t < 0) t += gw;
+    if (++rot == gw) rot = 0;
+    const uint32_t wbase = ring_s + s * a.slot_bytes + gid * pitch + 16 * r;
+    const int gs0 = c * (C >> 4);  // 64-byte step index of the chunk's first step
+    for (; t < nsteps; t += gw) {
+      uint4 wa[NT], wb[NT];
+#pragma unroll
+      for (int u = 0; u < NT; ++u) {
+        wa[u] = lds128(wbase + u * 16 * pitch + 64 * t);
+        wb[u] = lds128(wbase + u * 16 * pitch + 8 * pitch + 64 * t);
+      }
+      // Lanes of tokens >= T read another token's activations: they only feed accumulator
+      // columns that are never used.
+      uint4 xa[4], xb[4];
+      if (XSM) {
+        const uint32_t xo = 256u * (gs0 + t);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          xa[g] = lds128(xs_a + xo + 64 * g);
+          if (TG > 1) xb[g] = lds128(xs_b + xo + 64 * g);
+        }
+      } else {
+        // Weight bytes past the row end are zero (TMA fill); the activations there lie past
+        // the row in global memory, so those lanes read the row's first bytes instead.
+        const long long xo = 64 * t + 16 * r < cbytes ? 256LL * (gs0 + t) : 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          xa[g] = *reinterpret_cast<const uint4*>(xg_a + xo + 32 * g);
+          if (TG > 1) xb[g] = *reinterpret_cast<const uint4*>(xg_b + xo + 32 * g);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t m = 0x03030303u << (6 - 2 * g);
+#pragma unroll
+        for (int u = 0; u < NT; ++u) {
+          const uint32_t a0 = wa[u].x & m, a1 = wb[u].x & m, a2 = wa[u].y & m, a3 = wb[u].y & m;
+          const uint32_t a4 = wa[u].z & m, a5 = wb[u].z & m, a6 = wa[u].w & m, a7 = wb[u].w & m;
+          mma_u8s8(f[u][0][g], a0, a1, a2, a3, xa[g].x, xa[g].y);
+          mma_u8s8(f[u][0][g], a4, a5, a6, a7, xa[g].z, xa[g].w);
+          if (TG > 1) {
+            mma_u8s8(f[u][TG - 1][g], a0, a1, a2, a3, xb[g].x, xb[g].y);
+            mma_u8s8(f[u][TG - 1][g], a4, a5, a6, a7, xb[g].z, xb[g].w);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_count(bar0 + 8u * (a.n_slots + s), (uint32_t)ng);
+    if (last) {
+      int* at = acc + tl * NT * GEMV_ROWS * T;
+#pragma unroll
+      for (int u = 0; u < NT; ++u)
+#pragma unroll
+        for (int tg = 0; tg < TG; ++tg)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int v = (f[u][tg][0][i] >> 6) + (f[u][tg][1][i] >> 4) + (f[u][tg][2][i] >> 2) + f[u][tg][3][i];
+            const int row = gid + ((i & 2) ? 8 : 0), tok = tg * 8 + 2 * r + (i & 1);
+            if (tok < T) atomicAdd(at + (u * GEMV_ROWS + row) * T + tok, v);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) f[u][tg][g][i] = 0;
+          }
+    }
+  }
+  // past the phase's last stage
+  slot += sc.R * ng * nch + rem_len_total - done;
+  seq += sc.R * ng * nch + rem_len_total;
+  while (slot >= a.n_slots) {
+    slot -= a.n_slots;
+    par ^= 1u;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int TG>
 __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant__ EngArgs args,
@@ -381,13 +643,14 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   __shared__ float s_loc_s[ENG_MAX_T];
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
   __shared__ float s_beta[ENG_MAX_PHASES][4];
+  volatile __shared__ int s_slot_tag[ENG_MAX_SLOTS];  // stage index the producer last put in each slot
 
   // TMA boxes land 1024-byte aligned.
   uint8_t* ring = smem + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
   const uint32_t bar0 = smem_addr(ring + a.n_slots * a.slot_bytes);
   int* acc = reinterpret_cast<int*>(ring + a.n_slots * a.slot_bytes + 16 * a.n_slots);
-  int8_t* qs = reinterpret_cast<int8_t*>(acc + a.acc_ints);
-  float* xs = reinterpret_cast<float*>(qs + a.qs_bytes);  // fp32 staging of one activation row
+  int8_t* qs = reinterpret_cast<int8_t*>(acc + a.acc_ints);  // activations, layout eng_perm
+  float* xs = reinterpret_cast<float*>(qs + a.qs_bytes);     // fp32 staging of one activation row
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (a.n_slots + s); };
 
@@ -397,7 +660,8 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.n_slots; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), ENG_CONS_WARPS);
+      mbar_init(empty(s), ENG_CONS_WARPS);  // each warp of the owning group arrives with count ng
+      s_slot_tag[s] = -1;
     }
     s_abort = 0;
     fence_mbar_init();
@@ -425,44 +689,45 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     n0 = (tile - p.t[ti].tile_begin) * GEMV_ROWS;
     nrows = min(GEMV_ROWS, p.t[ti].N - n0);
   };
-  // The stage group starting at tile g0: up to m_tiles tiles of the same tensor, ending at
-  // g1; n0 is its first row.
-  auto group = [&](const EngPhase& p, int g0, int te, int& ti, int& n0, int& g1) {
-    int nr;
-    locate(p, g0, ti, n0, nr);
-    const int tensor_end = (p.kind == PH_GEMV && ti + 1 < p.n_tensors) ? p.t[ti + 1].tile_begin : p.n_tiles;
-    g1 = min(min(te, tensor_end), g0 + p.m_tiles);
-  };
 
   if (warp == ENG_CONS_WARPS) {
     // ------------------------------------------------------------ producer
-    // One elected lane per tensor issues a 2-D TMA box per stage (no multicast).
-    int st = 0;
+    // Lane u < NT issues the box of tensor u of each stage (no multicast).
+    int slot = 0, seq = 0;
+    uint32_t par = 0;
     for (int pi = 0; pi < a.n_phases && !s_abort; ++pi) {
       const EngPhase& p = a.ph[pi];
       if (p.kind == PH_QUANT) continue;
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
+      const uint32_t box_bytes = 64u * (uint32_t)p.chunk_words;
       int tb, te;
       tile_range(p, tb, te);
-      for (int g0 = tb; g0 < te && !s_abort;) {
-        int ti, n0, g1;
-        group(p, g0, te, ti, n0, g1);
-        for (int c = 0; c < p.n_chunks; ++c, ++st) {
-          const int slot = st % a.n_slots;
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait_bounded(empty(slot), ((st / a.n_slots) & 1) ^ 1);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) {
-            s_abort = 1;
-            break;
-          }
-          if (lane == 0) mbar_arrive_expect_tx(full(slot), (uint32_t)p.stage_bytes);
-          __syncwarp();
-          if (lane < NT)
-            tma_load_2d(smem_addr(ring + slot * a.slot_bytes + lane * p.box_rows * p.chunk_words * 4),
-                            &maps.m[pi][NT == 2 ? lane : ti], c * p.chunk_words, n0, full(slot));
+      EngSched sc(te - tb, p.n_chunks);
+      int grp, tl, c;
+      bool last;
+      while (!s_abort && sc.next(grp, tl, c, last)) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(empty(slot), par ^ 1u);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          s_abort = 1;
+          break;
         }
-        g0 = g1;
+        int ti, n0, nr;
+        locate(p, tb + tl, ti, n0, nr);
+        if (lane == 0) {
+          s_slot_tag[slot] = seq;
+          mbar_arrive_expect_tx(full(slot), (uint32_t)p.stage_bytes);
+        }
+        __syncwarp();
+        if (lane < NT)
+          tma_load_2d(smem_addr(ring + slot * a.slot_bytes + lane * box_bytes), &maps.m[pi][NT == 2 ? lane : ti],
+                      c * p.chunk_words, n0, full(slot));
+        ++seq;
+        if (++slot == a.n_slots) {
+          slot = 0;
+          par ^= 1u;
+        }
       }
     }
   } else {
@@ -470,9 +735,11 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     const int gid = lane >> 2, r = lane & 3;
     const int t_a = gid, t_b = 8 + gid;
     pdl_wait();  // activations and workspace belong to the previous kernel until now
-    int st = 0;
-    // Every branch that leaves the phase loop is taken by all 256 consumer threads
-    // together (barrier.red.or consensus), so no thread is left at a named barrier.
+    int slot = 0;       // ring position of the next stage
+    uint32_t par = 0;   // and the phase parity of its barriers
+    int seq = 0;        // index of the phase's first stage in the producer's sequence
+    // Every branch that leaves the phase loop is taken by all consumer threads together
+    // (barrier.red.or consensus), so no thread is left at a named barrier.
     for (int pi = 0; pi < a.n_phases; ++pi) {
       const EngPhase& p = a.ph[pi];
       if (named_sync_or(1, ENG_CONS, s_abort != 0)) break;
@@ -486,164 +753,85 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
       if (p.kind == PH_QUANT) {
         for (int t = blockIdx.x; t < T; t += gridDim.x) {
           quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
-                    p.gain, a.eps, p.q + (long long)t * p.K, p.s + t, p.sq + t, s_red, xs);
+                    p.gain, a.eps, p.q + (long long)t * p.K, false, p.s + t, p.sq + t, s_red, xs);
         }
         if (p.arrive_barrier >= 0) grid_arrive(a.counters + p.arrive_barrier);
         continue;
       }
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-      const int row_bytes = p.K >> 2;
       int tb, te;
       tile_range(p, tb, te);
-      // Activations of this phase.
+      const int nt = te - tb;
+      const int xp = eng_x_pitch(p.K), K16 = p.K >> 4;
+      // Activations of this phase: in shared memory (layout eng_perm) when they fit, else
+      // read in plain order from global memory.
       const bool local = p.src == SRC_LOCAL;
+      const bool xsm = local || T * xp <= a.qs_bytes;
       if (local) {
         for (int t = 0; t < T; ++t) {
           quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
-                    p.gain, a.eps, qs + t * p.K, s_loc_s + t, s_loc_sq + t, s_red, xs);
+                    p.gain, a.eps, qs + t * xp, true, s_loc_s + t, s_loc_sq + t, s_red, xs);
         }
-        if (blockIdx.x == 0 && p.q != nullptr) {  // one copy for callers that read the intermediates
-          for (int i = threadIdx.x; i < T * p.K / 16; i += ENG_CONS)
-            reinterpret_cast<uint4*>(p.q)[i] = reinterpret_cast<const uint4*>(qs)[i];
+        if (blockIdx.x == 0 && p.q != nullptr) {  // one plain-order copy for callers that read the intermediates
+          for (int i = threadIdx.x; i < T * K16; i += ENG_CONS) {
+            const int t = i / K16, k = (i - t * K16) * 16;
+            *reinterpret_cast<uint4*>(p.q + (long long)t * p.K + k) =
+                *reinterpret_cast<const uint4*>(qs + t * xp + eng_perm(k));
+          }
           if (threadIdx.x < T) {
             p.s[threadIdx.x] = s_loc_s[threadIdx.x];
             p.sq[threadIdx.x] = s_loc_sq[threadIdx.x];
           }
         }
+      } else if (xsm) {
+        // Written by this launch's QUANT phase or by the previous kernel: read past L1.
+        for (int i = threadIdx.x; i < T * K16; i += ENG_CONS) {
+          const int t = i / K16, k = (i - t * K16) * 16;
+          *reinterpret_cast<uint4*>(qs + t * xp + eng_perm(k)) =
+              __ldcg(reinterpret_cast<const uint4*>(p.q + (long long)t * p.K + k));
+        }
       }
-      for (int i = threadIdx.x; i < (te - tb) * NT * 256; i += ENG_CONS) acc[i] = 0;
+      for (int i = threadIdx.x; i < nt * NT * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
       cons_sync();
 
-      // Products: the global step index g runs over (stage, 64-byte step); warp w takes
-      // the steps with g % 8 == w, so short stages still use every warp.
-      int f[2][TG][4][4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) f[u][tg][g][i] = 0;
-      int gstep = 0;
-      const int W = p.K >> 4;  // 32-bit words per row
-      for (int g0 = tb; g0 < te && !s_abort;) {
-        int ti, n0, g1;
-        group(p, g0, te, ti, n0, g1);
-        const int N = p.t[ti].N;
-        for (int c = 0; c < p.n_chunks; ++c, ++st) {
-          const int slot = st % a.n_slots;
-          const int cb = 4 * min(p.chunk_words, W - c * p.chunk_words);  // bytes of this chunk per row
-          const int nsteps = (cb + 63) >> 6;
-          const int pitch = 4 * p.chunk_words;                          // row pitch of the box
-          const uint8_t* sbase = ring + slot * a.slot_bytes;
-          bool waited = false;
-          if (s_abort) break;
-          for (int j = 0; j < g1 - g0; ++j) {
-            const int first = (warp - gstep % ENG_CONS_WARPS + ENG_CONS_WARPS) % ENG_CONS_WARPS;
-            gstep += nsteps;
-            if (first >= nsteps) continue;
-            if (!waited) {
-              if (!mbar_wait_bounded(full(slot), (st / a.n_slots) & 1)) {
-                s_abort = 1;
-                break;
-              }
-              waited = true;
-            }
-            const int nrows = min(GEMV_ROWS, N - n0 - GEMV_ROWS * j);
-            for (int step = first; step < nsteps; step += ENG_CONS_WARPS) {
-              const int boff = 64 * step + 16 * r;
-              const bool valid = boff < cb;
-              uint4 wa[2], wb[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                if (u < NT) {
-                  const uint8_t* rb = sbase + (u * p.box_rows + GEMV_ROWS * j) * pitch + boff;
-                  wa[u] = (valid && gid < nrows) ? *reinterpret_cast<const uint4*>(rb + gid * pitch)
-                                                 : make_uint4(0, 0, 0, 0);
-                  wb[u] = (valid && gid + 8 < nrows) ? *reinterpret_cast<const uint4*>(rb + (gid + 8) * pitch)
-                                                     : make_uint4(0, 0, 0, 0);
-                }
-              }
-              const int kb = 4 * (c * 4 * p.chunk_words + 64 * step) + 128 * (r >> 1) + 16 * (r & 1);
-              uint4 xa[4], xb[4];
-#pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const uint4 z = make_uint4(0, 0, 0, 0);
-                if (local) {
-                  xa[g] = (valid && t_a < T) ? *reinterpret_cast<const uint4*>(qs + t_a * p.K + kb + 32 * g) : z;
-                  xb[g] = (TG > 1 && valid && t_b < T) ? *reinterpret_cast<const uint4*>(qs + t_b * p.K + kb + 32 * g)
-                                                       : z;
-                } else {
-                  // Plain (L1-cached) loads: this SM has not read these lines before in this
-                  // launch (L1 starts empty), and they were complete when the phase's grid
-                  // barrier was passed.
-                  xa[g] = (valid && t_a < T) ? *reinterpret_cast<const uint4*>(p.q + (long long)t_a * p.K + kb + 32 * g)
-                                             : z;
-                  xb[g] = (TG > 1 && valid && t_b < T)
-                              ? *reinterpret_cast<const uint4*>(p.q + (long long)t_b * p.K + kb + 32 * g)
-                              : z;
-                }
-              }
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                if (u < NT) {
-#pragma unroll
-                  for (int g = 0; g < 4; ++g) {
-                    const uint32_t m = 0x03030303u << (6 - 2 * g);
-                    mma_u8s8(f[u][0][g], wa[u].x & m, wb[u].x & m, wa[u].y & m, wb[u].y & m, xa[g].x, xa[g].y);
-                    mma_u8s8(f[u][0][g], wa[u].z & m, wb[u].z & m, wa[u].w & m, wb[u].w & m, xa[g].z, xa[g].w);
-                    if (TG > 1) {
-                      mma_u8s8(f[u][TG - 1][g], wa[u].x & m, wb[u].x & m, wa[u].y & m, wb[u].y & m, xb[g].x, xb[g].y);
-                      mma_u8s8(f[u][TG - 1][g], wa[u].z & m, wb[u].z & m, wa[u].w & m, wb[u].w & m, xb[g].z, xb[g].w);
-                    }
-                  }
-                }
-              }
-            }
-            // This warp's part of tile g0 + j in this stage -> the tile's shared accumulator.
-            int* at = acc + (g0 + j - tb) * NT * 256;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              if (u < NT) {
-#pragma unroll
-                for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    const int v = (f[u][tg][0][i] >> 6) + (f[u][tg][1][i] >> 4) + (f[u][tg][2][i] >> 2) + f[u][tg][3][i];
-                    const int row = gid + ((i & 2) ? 8 : 0), tok = tg * 8 + 2 * r + (i & 1);
-                    if (tok < T && row < nrows) atomicAdd(at + u * 256 + row * 16 + tok, v);
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) f[u][tg][g][i] = 0;
-                  }
-              }
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(empty(slot));
-        }
-        g0 = g1;
+      {
+        const uint32_t qs_s = smem_addr(qs);
+        const int ta = min(t_a, T - 1), tb2 = min(t_b, T - 1);
+        const uint32_t xs_a = qs_s + ta * xp + 16 * r, xs_b = qs_s + tb2 * xp + 16 * r;
+        const int8_t* xg_a = p.q + (long long)ta * p.K + 128 * (r >> 1) + 16 * (r & 1);
+        const int8_t* xg_b = p.q + (long long)tb2 * p.K + 128 * (r >> 1) + 16 * (r & 1);
+        const uint32_t ring_s = smem_addr(ring);
+#define ENG_PRODUCTS(NTV, XSMV)                                                                              \
+  eng_phase_products<TG, NTV, XSMV>(a, p, nt, ring_s, bar0, s_slot_tag, seq, slot, par, acc, xs_a, xs_b, xg_a, \
+                                    xg_b)
+        bool ok;
+        if (NT == 2)
+          ok = xsm ? ENG_PRODUCTS(2, true) : ENG_PRODUCTS(2, false);
+        else
+          ok = xsm ? ENG_PRODUCTS(1, true) : ENG_PRODUCTS(1, false);
+#undef ENG_PRODUCTS
+        if (!ok) s_abort = 1;
       }
       if (named_sync_or(1, ENG_CONS, s_abort != 0)) break;
       // Epilogue of this phase's tiles.
-      const int n_out = (te - tb) * GEMV_ROWS * T;
+      const int n_out = nt * GEMV_ROWS * T;
       for (int idx = threadIdx.x; idx < n_out; idx += ENG_CONS) {
-        const int tl = idx / (GEMV_ROWS * T), rem = idx % (GEMV_ROWS * T);
-        const int t = rem / GEMV_ROWS, row = rem % GEMV_ROWS;
+        const int tl2 = idx / (GEMV_ROWS * T), rem = idx - tl2 * (GEMV_ROWS * T);
+        const int t = rem / GEMV_ROWS, row = rem - t * GEMV_ROWS;
         int ti, n0, nrows;
-        locate(p, tb + tl, ti, n0, nrows);
+        locate(p, tb + tl2, ti, n0, nrows);
         if (row >= nrows) continue;
         const long long n = n0 + row;
         const int N = p.t[ti].N;
         const int sq = local ? s_loc_sq[t] : __ldcg(p.sq + t);
         const float sx = local ? s_loc_s[t] : __ldcg(p.s + t);
-        const int* at = acc + tl * NT * 256;
-        const int accA = at[row * 16 + t] - sq;
+        const int* at = acc + tl2 * NT * GEMV_ROWS * T;
+        const int accA = at[row * T + t] - sq;
         const float betaA = s_beta[pi][ti];
         const float vA = dequant(accA, __fdiv_rn(betaA, sx));
         if (NT == 2) {
           const float betaU = s_beta[pi][1];
-          const int accU = at[256 + row * 16 + t] - sq;
+          const int accU = at[(GEMV_ROWS + row) * T + t] - sq;
           const float vU = dequant(accU, __fdiv_rn(betaU, sx));
           p.h[(long long)t * N + n] = ffn_act(vA, vU, p.act);
         } else {
@@ -654,7 +842,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
       if (p.arrive_barrier >= 0)
         grid_arrive(a.counters + p.arrive_barrier);
       else
-        cons_sync();  // acc and the local activations are reused by the next phase
+        cons_sync();  // acc and the staged activations are reused by the next phase
     }
   }
 
