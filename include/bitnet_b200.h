@@ -137,7 +137,8 @@ size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I);
 /* Byte offsets inside that workspace, so that a caller can read the intermediates after
  * a call: off[0] q_x int8 [T,H], off[1] s_x fp32 [T], off[2] sum_x int32 [T],
  * off[3] h fp32 [T,I], off[4] q_h int8 [T,I], off[5] s_h fp32 [T], off[6] sum_h int32 [T],
- * off[7] 256 bytes of grid-barrier counters.  `off` is a HOST array of 8 entries.
+ * off[7] 256 bytes of grid-barrier counters, followed by the decode engine's per-CTA
+ * partial reductions (no layout promised).  `off` is a HOST array of 8 entries.
  * Returns BITNET_ERR_SHAPE on invalid sizes. */
 bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size_t* off);
 

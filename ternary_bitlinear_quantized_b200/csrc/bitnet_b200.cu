@@ -351,13 +351,14 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   bool multi = a.n_phases > 1;
   int max_tiles = 1;
   for (int i = 0; i < a.n_phases; ++i)
-    if (a.ph[i].kind != PH_QUANT && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
-  const int grid = multi ? sms : (max_tiles < sms ? max_tiles : sms);
+    if (ph_is_gemv(a.ph[i].kind) && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
+  const int gmax = sms < ENG_MAX_GRID ? sms : ENG_MAX_GRID;  // per-CTA partials are sized for ENG_MAX_GRID
+  const int grid = multi ? gmax : (max_tiles < gmax ? max_tiles : gmax);
   int acc_ints = 0, qs = 0, xs = 0;
   for (int i = 0; i < a.n_phases; ++i) {
     const EngPhase& p = a.ph[i];
-    if ((p.kind == PH_QUANT || p.src == SRC_LOCAL) && p.K > ENG_REG_MAX_K && p.K > xs) xs = p.K;
-    if (p.kind == PH_QUANT) continue;
+    if ((p.kind == PH_QUANT || (ph_is_gemv(p.kind) && p.src == SRC_LOCAL)) && p.K > ENG_REG_MAX_K && p.K > xs) xs = p.K;
+    if (!ph_is_gemv(p.kind)) continue;
     const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
     const int per = (p.n_tiles + grid - 1) / grid * NT * GEMV_ROWS * a.T;
     if (per > acc_ints) acc_ints = per;
@@ -387,7 +388,7 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < a.n_phases; ++i) {
     EngPhase& p = a.ph[i];
-    if (p.kind == PH_QUANT) continue;
+    if (!ph_is_gemv(p.kind)) continue;
     eng_chunks(p, slot_max);
     if (p.stage_bytes > slot) slot = p.stage_bytes;
     for (int u = 0; u < p.n_tensors; ++u)
@@ -574,14 +575,18 @@ bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size
   off[4] = o; o = align_up(o + (size_t)T * I);      // q_h
   off[5] = o; o = align_up(o + (size_t)T * 4);      // s_h
   off[6] = o; o = align_up(o + (size_t)T * 4);      // sum_h
-  off[7] = o;                                       // grid-barrier counters
+  off[7] = o;                                       // grid-barrier counters, then per-CTA partials
   return BITNET_OK;
 }
+
+// Per-CTA partial reductions of the distributed sub-norm after the counters: max [T][G]
+// fp32 and fixed-point sums [T][G] int64, G = ENG_MAX_GRID.
+static size_t ffn_partials_bytes(int64_t T) { return align_up((size_t)T * ENG_MAX_GRID * 4) + (size_t)T * ENG_MAX_GRID * 8; }
 
 size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I) {
   size_t off[FFN_WS_SLOTS];
   if (bitnet_ffn_workspace_offsets(T, H, I, off) != BITNET_OK) return 0;
-  return off[7] + ENG_COUNTER_BYTES;
+  return off[7] + ENG_COUNTER_BYTES + ffn_partials_bytes(T);
 }
 
 // Appends the FFN phases (x [T, H] -> out [T, H]) to an engine plan; `bar` is the next
@@ -613,20 +618,39 @@ static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32,
     gate_up.wait_barrier = qp.arrive_barrier;
   }
   gate_up.arrive_barrier = bar++;
-  ea.ph[ea.n_phases++] = gate_up;
   const int64_t nH[1] = {H};
   void* o[1] = {out};
   EngPhase down = eng_gemv((int)I, false, 1, &p_down, nH, o, nullptr, ot, act, nullptr);
   if (eng_local_ok(T, I)) {
+    ea.ph[ea.n_phases++] = gate_up;
     eng_src_local(down, h, 1, g_sub, q_h, s_h, sum_h);
     down.wait_barrier = gate_up.arrive_barrier;
   } else {
-    EngPhase qp = eng_quant(h, 1, (int)I, g_sub, q_h, s_h, sum_h);
-    qp.wait_barrier = gate_up.arrive_barrier;
-    qp.arrive_barrier = bar++;
-    ea.ph[ea.n_phases++] = qp;
+    // ffn_sub_norm spread over the grid: every CTA reduces the rows of h it produced.
+    float* pmax = reinterpret_cast<float*>(ws + off[7] + ENG_COUNTER_BYTES);
+    long long* psum = reinterpret_cast<long long*>(ws + off[7] + ENG_COUNTER_BYTES + align_up((size_t)T * ENG_MAX_GRID * 4));
+    gate_up.pmax = pmax;
+    ea.ph[ea.n_phases++] = gate_up;
+    EngPhase sp;
+    memset(&sp, 0, sizeof(sp));
+    sp.kind = PH_SUBNORM;
+    sp.K = (int)I;
+    sp.n_tiles = gate_up.n_tiles;
+    sp.x = h;
+    sp.x_f32 = 1;
+    sp.gain = g_sub;
+    sp.q = q_h;
+    sp.s = s_h;
+    sp.sq = sum_h;
+    sp.pmax = pmax;
+    sp.psum = psum;
+    sp.wait_barrier = gate_up.arrive_barrier;
+    sp.bar_a = bar++;
+    sp.bar_b = bar++;
+    sp.arrive_barrier = bar++;
+    ea.ph[ea.n_phases++] = sp;
     eng_src_global(down, q_h, s_h, sum_h);
-    down.wait_barrier = qp.arrive_barrier;
+    down.wait_barrier = sp.arrive_barrier;
   }
   ea.ph[ea.n_phases++] = down;
 }

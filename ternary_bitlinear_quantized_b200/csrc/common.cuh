@@ -9,6 +9,7 @@
 #include "../../include/bitnet_b200.h"
 
 #define BN_DEV __device__ __forceinline__
+#define BN_HOST_DEV __host__ __device__
 
 namespace bitnet {
 

@@ -6,7 +6,10 @@
 //             is either given (q, s_x, sum_q in global memory) or quantised by every CTA
 //             itself from the raw activations (RMSNorm + absmax int8 in registers);
 //   QUANT     RMSNorm + absmax int8 of a larger activation batch, tokens split over CTAs,
-//             written to global memory.
+//             written to global memory;
+//   SUBNORM   the FFN's ffn_sub_norm + absmax int8 of h, every row split over all CTAs:
+//             each CTA reduces the rows it produced in the gate/up phase, with grid
+//             barriers between the global max, the exact sum of squares and max |y|.
 //
 // A phase may arrive on a grid barrier after its epilogue (its outputs are complete
 // once every CTA has arrived) and may wait on one before it reads its inputs.  Arrival
@@ -45,7 +48,9 @@ constexpr int ENG_LOCAL_MAX_K = 28672;  // rows staged in shared memory as fp32 
 constexpr int ENG_MAX_T = 16;
 constexpr int ENG_MAX_SLOTS = 32;  // ring slots at most
 
-enum { PH_GEMV = 0, PH_GEMV_FFN = 1, PH_QUANT = 2 };
+enum { PH_GEMV = 0, PH_GEMV_FFN = 1, PH_QUANT = 2, PH_SUBNORM = 3 };
+BN_HOST_DEV inline bool ph_is_gemv(int kind) { return kind == PH_GEMV || kind == PH_GEMV_FFN; }
+constexpr int ENG_MAX_GRID = 256;  // CTAs at most (per-CTA partials in the workspace)
 enum { SRC_GLOBAL = 0, SRC_LOCAL = 1 };
 
 struct EngTensor {
@@ -69,6 +74,12 @@ struct EngPhase {
   int out_dtype, act;
   float* h;           // FFN output [T, N] fp32
   int wait_barrier, arrive_barrier;  // -1: none
+  // SUBNORM (and the GEMV_FFN phase before it): per-CTA partials [T][gridDim.x] of
+  // max |h| then max |y| (pmax) and of the fixed-point sum of h^2 (psum); the SUBNORM
+  // phase's two inner grid barriers.
+  float* pmax;
+  long long* psum;
+  int bar_a, bar_b;
   // Stage geometry: a stage is one 2-D TMA box per tensor of 16 rows (one tile) x
   // chunk_words 32-bit words (a K-chunk; chunk_words = 16 mod 32, so the rows of a box are
   // 64 mod 128 bytes apart); stage_bytes = tensors x 64 x chunk_words.
@@ -375,6 +386,149 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
   return ok;
 }
 
+// ------------------------------------------------------------------ distributed sub-norm
+// Per-token scratch of the SUBNORM phase in shared memory.
+struct SubScratch {
+  unsigned mx[ENG_MAX_T];  // max |h|, then max |y| (non-negative floats as bits)
+  unsigned my[ENG_MAX_T];
+  unsigned long long sum[ENG_MAX_T];
+  float inv[ENG_MAX_T];
+  float scale[ENG_MAX_T];
+  int sq[ENG_MAX_T];
+};
+
+// Grid barrier between two steps of a phase: arrive, wait for every CTA, and agree on the
+// outcome (false: a wait gave up).
+BN_DEV bool grid_step(unsigned* ctr) {
+  grid_arrive(ctr);
+  const bool ok = grid_wait(ctr, gridDim.x);
+  return !named_sync_or(1, ENG_CONS, !ok);
+}
+
+// ffn_sub_norm + absmax int8 of h [T, K] (fp32, plain order) into p.q / p.s / p.sq, every
+// row split over the grid: this CTA owns the 16-row tiles [tb, te) it produced in the
+// gate/up phase, whose epilogue left max |h| of those rows in p.pmax[t][cta].  The same
+// arithmetic as quant_row, with each reduction finished across the grid: max |h| ->
+// exponent e -> exact fixed-point sum of h^2 -> inv -> y = h * inv * g -> max |y| -> s_x
+// -> q.  Maxima and integer sums are order-free, so the result does not depend on the
+// split.  p.sq must be zero on entry (the kernel clears it before the gate/up phase).
+__device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, int tb, int te, unsigned* counters,
+                                         SubScratch& S) {
+  const int G = gridDim.x, K = p.K, tid = threadIdx.x, nt = te - tb;
+  const float* h = reinterpret_cast<const float*>(p.x);
+  if (tid < T) {
+    S.mx[tid] = S.my[tid] = 0u;
+    S.sum[tid] = 0ull;
+    S.sq[tid] = 0;
+  }
+  cons_sync();
+  for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.mx[i / G], __float_as_uint(__ldcg(p.pmax + i)));
+  cons_sync();
+  if (p.gain != nullptr) {
+    // exact fixed-point sum of h^2 over this CTA's rows
+    for (int i = tid; i < T * nt; i += ENG_CONS) {
+      const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
+      const float am = __uint_as_float(S.mx[t]);
+      if (am > 0.0f) {
+        const double p2e = pow2_f64(fixed_point_exponent(__dmul_rn((double)am, (double)am), K));
+        long long part = 0;
+#pragma unroll
+        for (int j = 0; j < GEMV_ROWS; j += 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const double d = (double)vv[k];
+            part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
+          }
+        }
+        atomicAdd(&S.sum[t], (unsigned long long)part);
+      }
+    }
+    cons_sync();
+    if (tid < T) p.psum[tid * G + blockIdx.x] = (long long)S.sum[tid];
+    if (!grid_step(counters + p.bar_a)) return false;
+    if (tid < T) S.sum[tid] = 0ull;
+    cons_sync();
+    for (int i = tid; i < T * G; i += ENG_CONS) atomicAdd(&S.sum[i / G], (unsigned long long)__ldcg(p.psum + i));
+    cons_sync();
+    if (tid < T) {
+      const float am = __uint_as_float(S.mx[tid]);
+      float ms = 0.0f;
+      if (am > 0.0f)
+        ms = fixed_point_mean((long long)S.sum[tid], fixed_point_exponent(__dmul_rn((double)am, (double)am), K), K);
+      S.inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    }
+    cons_sync();
+    // max |y| over this CTA's rows
+    for (int i = tid; i < T * nt; i += ENG_CONS) {
+      const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
+      const float inv = S.inv[t];
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < GEMV_ROWS; j += 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
+        const float4 g = __ldg(reinterpret_cast<const float4*>(p.gain + r0 + j));
+        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.x, inv), g.x)));
+        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.y, inv), g.y)));
+        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.z, inv), g.z)));
+        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.w, inv), g.w)));
+      }
+      atomicMax(&S.my[t], __float_as_uint(m));
+    }
+    cons_sync();
+    // every CTA has read max |h| before passing bar_a, so pmax can hold max |y| now
+    if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
+    if (!grid_step(counters + p.bar_b)) return false;
+    if (tid < T) S.my[tid] = 0u;
+    cons_sync();
+    for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.my[i / G], __float_as_uint(__ldcg(p.pmax + i)));
+    cons_sync();
+  } else {
+    if (tid < T) {
+      S.my[tid] = S.mx[tid];  // y = h
+      S.inv[tid] = 1.0f;
+    }
+    cons_sync();
+  }
+  if (tid < T) S.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(S.my[tid]), 1e-5f));
+  cons_sync();
+  // q of this CTA's rows, 16 bytes per tile row group
+  for (int i = tid; i < T * nt; i += ENG_CONS) {
+    const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
+    const float inv = S.inv[t], sc = S.scale[t];
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < GEMV_ROWS; j += 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
+      float y[4] = {v.x, v.y, v.z, v.w};
+      if (p.gain != nullptr) {
+        const float4 g = __ldg(reinterpret_cast<const float4*>(p.gain + r0 + j));
+        y[0] = __fmul_rn(__fmul_rn(v.x, inv), g.x);
+        y[1] = __fmul_rn(__fmul_rn(v.y, inv), g.y);
+        y[2] = __fmul_rn(__fmul_rn(v.z, inv), g.z);
+        y[3] = __fmul_rn(__fmul_rn(v.w, inv), g.w);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        int qv = __float2int_rn(__fmul_rn(y[k], sc));
+        qv = min(127, max(-128, qv));
+        sum += qv;
+        w[j >> 2] |= (uint32_t)(qv & 0xFF) << (8 * k);
+      }
+    }
+    *reinterpret_cast<uint4*>(p.q + (long long)t * K + r0) = make_uint4(w[0], w[1], w[2], w[3]);
+    atomicAdd(&S.sq[t], sum);
+  }
+  cons_sync();
+  if (tid < T) {
+    atomicAdd(p.sq + tid, S.sq[tid]);
+    if (blockIdx.x == 0) p.s[tid] = S.scale[tid];
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ stage schedule
 // A GEMV phase gives each CTA the tiles [tb, tb + nt) (16 weight rows; the tensors of a
 // group phase concatenated; for the FFN a tile is the gate and the up tile of the same
@@ -644,6 +798,8 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
   __shared__ float s_beta[ENG_MAX_PHASES][4];
   volatile __shared__ int s_slot_tag[ENG_MAX_SLOTS];  // stage index the producer last put in each slot
+  __shared__ SubScratch s_sub;
+  __shared__ unsigned s_hmax[ENG_MAX_T];  // max |h| of this CTA's rows (gate/up epilogue)
 
   // TMA boxes land 1024-byte aligned.
   uint8_t* ring = smem + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
@@ -669,7 +825,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   if (threadIdx.x < ENG_MAX_PHASES * 4) {  // per-tensor scales (weights: no dependency wait needed)
     const int pi = threadIdx.x >> 2, u = threadIdx.x & 3;
     float b = 0.0f;
-    if (pi < a.n_phases && a.ph[pi].kind != PH_QUANT && u < a.ph[pi].n_tensors) {
+    if (pi < a.n_phases && ph_is_gemv(a.ph[pi].kind) && u < a.ph[pi].n_tensors) {
       const EngTensor& t = a.ph[pi].t[u];
       b = __ldg(reinterpret_cast<const float*>(t.packed + (long long)t.N * (a.ph[pi].K >> 2)));
     }
@@ -697,7 +853,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     uint32_t par = 0;
     for (int pi = 0; pi < a.n_phases && !s_abort; ++pi) {
       const EngPhase& p = a.ph[pi];
-      if (p.kind == PH_QUANT) continue;
+      if (!ph_is_gemv(p.kind)) continue;
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
       const uint32_t box_bytes = 64u * (uint32_t)p.chunk_words;
       int tb, te;
@@ -738,6 +894,11 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     int slot = 0;       // ring position of the next stage
     uint32_t par = 0;   // and the phase parity of its barriers
     int seq = 0;        // index of the phase's first stage in the producer's sequence
+    // The SUBNORM phases accumulate sum_q with atomics: clear it before any CTA can get
+    // there (the grid barrier of the gate/up phase comes first).
+    if (blockIdx.x == 0 && threadIdx.x < T)
+      for (int i = 0; i < a.n_phases; ++i)
+        if (a.ph[i].kind == PH_SUBNORM) a.ph[i].sq[threadIdx.x] = 0;
     // Every branch that leaves the phase loop is taken by all consumer threads together
     // (barrier.red.or consensus), so no thread is left at a named barrier.
     for (int pi = 0; pi < a.n_phases; ++pi) {
@@ -756,6 +917,16 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
                     p.gain, a.eps, p.q + (long long)t * p.K, false, p.s + t, p.sq + t, s_red, xs);
         }
         if (p.arrive_barrier >= 0) grid_arrive(a.counters + p.arrive_barrier);
+        continue;
+      }
+      if (p.kind == PH_SUBNORM) {
+        int tb0, te0;
+        tile_range(p, tb0, te0);
+        if (!eng_subnorm(p, T, a.eps, tb0, te0, a.counters, s_sub)) {
+          s_abort = 1;
+          break;
+        }
+        grid_arrive(a.counters + p.arrive_barrier);
         continue;
       }
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
@@ -792,6 +963,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         }
       }
       for (int i = threadIdx.x; i < nt * NT * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
+      if (threadIdx.x < T) s_hmax[threadIdx.x] = 0u;
       cons_sync();
 
       {
@@ -833,11 +1005,17 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
           const float betaU = s_beta[pi][1];
           const int accU = at[(GEMV_ROWS + row) * T + t] - sq;
           const float vU = dequant(accU, __fdiv_rn(betaU, sx));
-          p.h[(long long)t * N + n] = ffn_act(vA, vU, p.act);
+          const float hv = ffn_act(vA, vU, p.act);
+          p.h[(long long)t * N + n] = hv;
+          if (p.pmax != nullptr) atomicMax(&s_hmax[t], __float_as_uint(fabsf(hv)));
         } else {
           store_out(p.t[ti].out, p.out_dtype, (long long)t * N + n, vA);
           if (p.t[ti].acc_debug) p.t[ti].acc_debug[(long long)t * N + n] = accA;
         }
+      }
+      if (p.pmax != nullptr) {  // max |h| of this CTA's rows, for the SUBNORM phase
+        cons_sync();
+        if (threadIdx.x < T) p.pmax[threadIdx.x * gridDim.x + blockIdx.x] = __uint_as_float(s_hmax[threadIdx.x]);
       }
       if (p.arrive_barrier >= 0)
         grid_arrive(a.counters + p.arrive_barrier);

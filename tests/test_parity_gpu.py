@@ -174,6 +174,29 @@ def test_ffn_block_parity(act, T, H, I):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("T,H,I", [(1, 512, 9216), (4, 256, 8320)])
+def test_ffn_block_distributed_sub_norm_without_gain_twice(T, H, I):
+    """The decode path spreads ffn_sub_norm over all CTAs when h is too long to quantise in
+    every CTA; here with ffn_sub_norm switched off (y = h) and the workspace reused."""
+    sh = workloads.BlockShape("ffn-nog", hidden=H, n_q=H, n_kv=H, inter=I, act="relu2")
+    d = workloads.block_inputs(sh, T, T + I, ffn_only=True)
+    pr = {nm: O.pack_i2s(d["W_" + nm].numpy()) for nm in ("gate", "up", "down")}
+    pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
+    ws = torch.zeros(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
+    ref, mid = O.ffn_block(bf16_to_np(d["x"]), d["g_ffn_norm"].numpy(), pr["gate"], pr["up"], None, pr["down"], H, I,
+                           "relu2", 1e-6, "bf16", return_intermediates=True)
+    off = tb.ffn_workspace_offsets(T, H, I)
+    for _ in range(2):
+        out = tb.ffn_block(d["x"].to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], None, pg["down"], I,
+                           tb.RELU2, 1e-6, torch.bfloat16, ws=ws)
+        torch.cuda.synchronize()
+        wsn = ws.cpu().numpy()
+        assert np.array_equal(wsn[off[4]:off[4] + T * I].view(np.int8).reshape(T, I), mid["q_h"])
+        assert np.array_equal(wsn[off[6]:off[6] + T * 4].view(np.int32), mid["sum_h"])
+        assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
+    assert tb.device_status() == 0
+
+
 def test_ffn_block_fp32_io():
     out, _, ref, _, dt = run_ffn(2, 384, 512, "silu", seed=5, out_dtype=torch.float32, x_dtype=torch.float32)
     assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
