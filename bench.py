@@ -121,8 +121,8 @@ def source_sha(files):
 
 
 def stored_traffic(kernel_key: str, sha: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it
-    was taken on the current kernel source."""
+    """DRAM bytes per launch of the dominant kernel ("<kernel> @ <workload>") from the
+    committed ncu summary, if it was taken on the current kernel source."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             d = json.load(f)
@@ -488,14 +488,14 @@ def main():
     if decode:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": stored_traffic(label, source_sha(kernel_files)), "kernel": label,
+                "traffic": stored_traffic(f"{label} @ {args.workload}", source_sha(kernel_files)), "kernel": label,
                 "bytes_per_launch": dom_bytes, "launch_us": dom_ms * 1e3,
                 "peak_source": f"{src} hbm_gbs (copy bandwidth, burst)"}
     else:
         achieved = dom_ops / (dom_ms / 1e3) / 1e12
         int8_peak = bf16 * 2.0  # dense int8 = 2x dense bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
         roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak,
-                "traffic": stored_traffic(label, source_sha(kernel_files)), "kernel": label,
+                "traffic": stored_traffic(f"{label} @ {args.workload}", source_sha(kernel_files)), "kernel": label,
                 "ops_per_launch": dom_ops, "launch_us": dom_ms * 1e3,
                 "peak_source": f"{src} bf16_tflops x 2 (nominal int8/bf16 ratio)"}
 
