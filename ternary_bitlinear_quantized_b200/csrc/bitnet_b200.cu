@@ -127,23 +127,25 @@ static bool make_map_u32(CUtensorMap* m, const void* base, uint64_t cols, uint64
 static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* gain, float eps, int64_t T, int64_t K,
                                    int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
   if (T == 0) return BITNET_OK;
-  // Rows of up to 8192 values (K a multiple of 8, 16-byte aligned rows): values in registers.
+  // Rows of up to 8192 values (K a multiple of 8, 16-byte aligned rows): values in registers,
+  // one to four warps per row.
   const size_t esz_r = xt == BITNET_BF16 ? 2 : 4;
-  if (K <= 4 * 8 * QR_THREADS && K % 8 == 0 && aligned16(x) && aligned16(q) && (K * esz_r) % 16 == 0) {
-    const int ng = K <= 2048 ? 1 : (K <= 4096 ? 2 : 4);
+  if (K <= 4 * 2048 && K % 8 == 0 && aligned16(x) && aligned16(q) && (K * esz_r) % 16 == 0) {
+    const int w = K <= 2048 ? 1 : (K <= 4096 ? 2 : 4);
+    const unsigned grid = (unsigned)((T + QW_THREADS / 32 / w - 1) / (QW_THREADS / 32 / w));
     cudaError_t e;
     if (xt == BITNET_BF16) {
-      auto* kern = ng == 1 ? k_rmsnorm_quant_regs<__nv_bfloat16, 1>
-                           : (ng == 2 ? k_rmsnorm_quant_regs<__nv_bfloat16, 2> : k_rmsnorm_quant_regs<__nv_bfloat16, 4>);
-      e = launch(kern, dim3((unsigned)T), dim3(QR_THREADS), 0, s, true, reinterpret_cast<const __nv_bfloat16*>(x), gain,
-                 eps, (int)K, q, s_x, sum_q);
+      auto* kern = w == 1 ? k_rmsnorm_quant_warps<__nv_bfloat16, 1>
+                          : (w == 2 ? k_rmsnorm_quant_warps<__nv_bfloat16, 2> : k_rmsnorm_quant_warps<__nv_bfloat16, 4>);
+      e = launch(kern, dim3(grid), dim3(QW_THREADS), 0, s, true, reinterpret_cast<const __nv_bfloat16*>(x), gain, eps,
+                 (int)T, (int)K, q, s_x, sum_q);
     } else {
-      auto* kern = ng == 1 ? k_rmsnorm_quant_regs<float, 1>
-                           : (ng == 2 ? k_rmsnorm_quant_regs<float, 2> : k_rmsnorm_quant_regs<float, 4>);
-      e = launch(kern, dim3((unsigned)T), dim3(QR_THREADS), 0, s, true, reinterpret_cast<const float*>(x), gain, eps,
+      auto* kern = w == 1 ? k_rmsnorm_quant_warps<float, 1>
+                          : (w == 2 ? k_rmsnorm_quant_warps<float, 2> : k_rmsnorm_quant_warps<float, 4>);
+      e = launch(kern, dim3(grid), dim3(QW_THREADS), 0, s, true, reinterpret_cast<const float*>(x), gain, eps, (int)T,
                  (int)K, q, s_x, sum_q);
     }
-    if (e != cudaSuccess) return cuda_fail(e, "k_rmsnorm_quant_regs");
+    if (e != cudaSuccess) return cuda_fail(e, "k_rmsnorm_quant_warps");
     return BITNET_OK;
   }
   int threads = (int)((K / 8 + 31) / 32 * 32);

@@ -153,49 +153,53 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
   quantise_staged_row(xs, K, gain, eps, q + t * K, s_x + t, sum_q + t, vec != 0, red, amax);
 }
 
-// The same arithmetic for rows of K <= 2048 * NG values held in registers by 256 threads
-// (thread i owns elements 8(i + 256 j) .. +7, j < NG), so a CTA reads its row once and
-// several tokens fit on one SM.  Reductions use one barrier each (two scratch halves used
-// in turn).
-constexpr int QR_THREADS = 256;
-constexpr int QR_WARPS = QR_THREADS / 32;
+// The same arithmetic with W warps per row (W = 1, 2 or 4) and 8 / W rows per 256-thread
+// CTA, for rows of K <= 2048 W values (K a multiple of 8, 16-byte aligned rows).  Lane l of
+// the row's warp `rank` holds elements 8 (l + 32 (rank + W j)) .. +7, j < 8, in registers, so
+// the row is read once; the reductions are warp shuffles, joined across the W warps by one
+// named barrier each (two scratch halves used in turn).  Many rows are in flight per SM,
+// which hides the latency of the loads and of the reduction chain.
+constexpr int QW_THREADS = 256;
+constexpr int QW_GROUPS = 8;
 
-template <typename T>
-BN_DEV T qr_reduce(T v, T* scratch, int& flip, bool is_max) {
+template <int W, typename T, typename Op>
+BN_DEV T qw_reduce(T v, T* slots, int& flip, int bar_id, int rank, Op op) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const T w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = is_max ? (v > w ? v : w) : v + w;
-  }
-  T* b = scratch + flip * QR_WARPS;
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (W == 1) return v;
+  T* b = slots + flip * W;
   flip ^= 1;
-  if ((threadIdx.x & 31) == 0) b[threadIdx.x >> 5] = v;
-  __syncthreads();
+  if ((threadIdx.x & 31) == 0) b[rank] = v;
+  named_sync(bar_id, 32 * W);
   T r = b[0];
 #pragma unroll
-  for (int w = 1; w < QR_WARPS; ++w) r = is_max ? (r > b[w] ? r : b[w]) : r + b[w];
+  for (int i = 1; i < W; ++i) r = op(r, b[i]);
   return r;
 }
 
-template <typename TIn, int NG>
-__global__ void __launch_bounds__(QR_THREADS) k_rmsnorm_quant_regs(const TIn* __restrict__ x,
-                                                                  const float* __restrict__ gain, float eps, int K,
-                                                                  int8_t* __restrict__ q, float* __restrict__ s_x,
-                                                                  int32_t* __restrict__ sum_q) {
-  __shared__ float redf[2 * QR_WARPS];
-  __shared__ long long redl[2 * QR_WARPS];
-  __shared__ int redi[2 * QR_WARPS];
-  int ff = 0, fl = 0, fi = 0;
-  const long long t = blockIdx.x;
-  const int tid = threadIdx.x;
+template <typename TIn, int W>
+__global__ void __launch_bounds__(QW_THREADS) k_rmsnorm_quant_warps(const TIn* __restrict__ x,
+                                                                   const float* __restrict__ gain, float eps, int T,
+                                                                   int K, int8_t* __restrict__ q,
+                                                                   float* __restrict__ s_x, int32_t* __restrict__ sum_q) {
+  constexpr int ROWS = QW_THREADS / 32 / W;
+  __shared__ float redf[ROWS][2 * W];
+  __shared__ long long redl[ROWS][2 * W];
+  __shared__ int redi[ROWS][2 * W];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rr = warp / W, rank = warp - rr * W;
+  const long long t = (long long)blockIdx.x * ROWS + rr;
   pdl_launch_dependents();
   pdl_wait();
+  if (t >= T) return;  // every warp of the row leaves together
+  const int bar = 1 + rr;
+  int ff = 0, fl = 0, fi = 0;
   const TIn* xr = x + t * K;
-  float v[NG][8];
+  float v[QW_GROUPS][8];
   float am = 0.0f;
 #pragma unroll
-  for (int j = 0; j < NG; ++j) {
-    const int k = 8 * (tid + QR_THREADS * j);
+  for (int j = 0; j < QW_GROUPS; ++j) {
+    const int k = 8 * (lane + 32 * (rank + W * j));
     if (k < K) {
       RowLoader<TIn>::load(xr + k, v[j]);
     } else {
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(QR_THREADS) k_rmsnorm_quant_regs(const TIn* __
 #pragma unroll
     for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[j][i]));
   }
-  am = qr_reduce(am, redf, ff, true);
+  am = qw_reduce<W>(am, &redf[rr][0], ff, bar, rank, MaxOp());
   float a = am;
   if (gain != nullptr) {
     float ms = 0.0f;
@@ -215,37 +219,40 @@ __global__ void __launch_bounds__(QR_THREADS) k_rmsnorm_quant_regs(const TIn* __
       const double p2e = pow2_f64(e);
       long long part = 0;
 #pragma unroll
-      for (int j = 0; j < NG; ++j)
-        if (8 * (tid + QR_THREADS * j) < K) {
+      for (int j = 0; j < QW_GROUPS; ++j)
+        if (8 * (lane + 32 * (rank + W * j)) < K) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const double d = (double)v[j][i];
             part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
           }
         }
-      ms = fixed_point_mean(qr_reduce(part, redl, fl, false), e, K);
+      ms = fixed_point_mean(qw_reduce<W>(part, &redl[rr][0], fl, bar, rank, AddOpLL()), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     float ay = 0.0f;
 #pragma unroll
-    for (int j = 0; j < NG; ++j) {
-      const int k = 8 * (tid + QR_THREADS * j);
+    for (int j = 0; j < QW_GROUPS; ++j) {
+      const int k = 8 * (lane + 32 * (rank + W * j));
       if (k < K) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain + k));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain + k + 4));
+        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          v[j][i] = __fmul_rn(__fmul_rn(v[j][i], inv), __ldg(gain + k + i));
+          v[j][i] = __fmul_rn(__fmul_rn(v[j][i], inv), g[i]);
           ay = fmaxf(ay, fabsf(v[j][i]));
         }
       }
     }
-    a = qr_reduce(ay, redf, ff, true);
+    a = qw_reduce<W>(ay, &redf[rr][0], ff, bar, rank, MaxOp());
   }
   const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
   int sum = 0;
   int8_t* qr = q + t * K;
 #pragma unroll
-  for (int j = 0; j < NG; ++j) {
-    const int k = 8 * (tid + QR_THREADS * j);
+  for (int j = 0; j < QW_GROUPS; ++j) {
+    const int k = 8 * (lane + 32 * (rank + W * j));
     if (k < K) {
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -258,8 +265,8 @@ __global__ void __launch_bounds__(QR_THREADS) k_rmsnorm_quant_regs(const TIn* __
       *reinterpret_cast<uint2*>(qr + k) = make_uint2(w[0], w[1]);
     }
   }
-  sum = qr_reduce(sum, redi, fi, false);
-  if (tid == 0) {
+  sum = qw_reduce<W>(sum, &redi[rr][0], fi, bar, rank, AddOpI());
+  if (rank == 0 && lane == 0) {
     s_x[t] = s;
     sum_q[t] = sum;
   }
