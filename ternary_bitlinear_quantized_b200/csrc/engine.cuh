@@ -35,6 +35,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "engine_sched.h"
 #include "gemv.cuh"
 
 namespace bitnet {
@@ -530,69 +531,8 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
 }
 
 // ------------------------------------------------------------------ stage schedule
-// A GEMV phase gives each CTA the tiles [tb, tb + nt) (16 weight rows; the tensors of a
-// group phase concatenated; for the FFN a tile is the gate and the up tile of the same
-// rows).  A stage is one tile x one K-chunk: one 2-D TMA box per tensor.  The consumer
-// warps form ng groups of ENG_CONS_WARPS / ng warps.  A group owns a tile for all of its
-// chunks, so its warps keep their partial sums in registers across the chunks and add
-// them to the tile's shared accumulator once.  Tiles are dealt to the groups in rounds of
-// ng; the tiles of a last, partial round are split by chunks between the groups.
-// Producer and consumers walk the same sequence with this iterator.
-BN_DEV int eng_groups(int nt) { return nt >= 5 ? 5 : (nt >= 3 ? 3 : 1); }
-
-struct EngSched {
-  int nch, ng, R, s, units, maxlen;
-  int a, b, q;
-  bool rem;
-  BN_DEV EngSched(int nt, int nch_) : nch(nch_), a(0), b(0), q(0), rem(false) {
-    ng = eng_groups(nt);
-    R = nt / ng;
-    const int left = nt - R * ng;
-    s = left == 0 ? 1 : (nch >= 2 ? min(ng / left, nch) : 1);
-    units = left * s;
-    maxlen = (nch + s - 1) / s;
-  }
-  // Next stage: owning group, tile (local index), chunk, and whether it is the last chunk
-  // of the group's share of the tile.  False at the end.
-  BN_DEV bool next(int& grp, int& tile, int& c, bool& last) {
-    while (true) {
-      if (!rem) {
-        if (a >= R) {
-          rem = true;
-          a = 0;
-          q = 0;
-          continue;
-        }
-        grp = q;
-        tile = a * ng + q;
-        c = b;
-        last = b == nch - 1;
-        if (++q == ng) {
-          q = 0;
-          if (++b == nch) {
-            b = 0;
-            ++a;
-          }
-        }
-        return true;
-      }
-      if (a >= maxlen || units == 0) return false;
-      const int u = q, i = a;
-      if (++q == units) {
-        q = 0;
-        ++a;
-      }
-      const int k = u % s, cb = nch * k / s, ce = nch * (k + 1) / s;
-      if (cb + i < ce) {
-        grp = u;
-        tile = R * ng + u / s;
-        c = cb + i;
-        last = c == ce - 1;
-        return true;
-      }
-    }
-  }
-};
+// EngSched / EngOwnStages (engine_sched.h): the producer walks the whole sequence, each
+// consumer group only its own stages.
 
 // Wait until the producer has tagged ring slot `tag` with stage `want` (bounded, like the
 // barrier waits).
@@ -637,50 +577,14 @@ __device__ __forceinline__ bool eng_phase_products(const EngArgs& a, const EngPh
       for (int g = 0; g < 4; ++g)
 #pragma unroll
         for (int i = 0; i < 4; ++i) f[u][tg][g][i] = 0;
-  // This group's stages, in sequence order: in the full rounds every ng-th stage (tile
-  // r * ng + my_grp, chunks 0 .. nch-1); in the last round unit my_grp, whose stage i sits
-  // at i * units + my_grp while every unit still has a chunk i (i < lmin), else after the
-  // units that do.  `pos` is the sequence index of the stage, `done` how far the ring
-  // position (slot, par) has been advanced.
+  // This group's stages in sequence order; `done` is how far the ring position (slot, par)
+  // has been advanced.
   const EngSched sc(nt, p.n_chunks);
-  const int nch = p.n_chunks;
-  int rot = 0, done = 0, rr = 0, cc = 0;
-  const int own_full = sc.R * nch;
-  int own_rem = 0, ucb = 0, lmin = 0, rank = 0;
-  if (my_grp < sc.units) {
-    const int k = my_grp % sc.s;
-    ucb = nch * k / sc.s;
-    own_rem = nch * (k + 1) / sc.s - ucb;
-    lmin = nch / sc.s;
-    for (int u = 0; u < my_grp; ++u) {
-      const int ku = u % sc.s;
-      if (nch * (ku + 1) / sc.s - nch * ku / sc.s > lmin) ++rank;
-    }
-  }
-  int rem_len_total = 0;  // stages of the last round
-  for (int u = 0; u < sc.units; ++u) {
-    const int ku = u % sc.s;
-    rem_len_total += nch * (ku + 1) / sc.s - nch * ku / sc.s;
-  }
-  for (int j = 0; j < own_full + own_rem; ++j) {
-    int pos, tl, c;
-    bool last;
-    if (j < own_full) {
-      c = cc;
-      tl = rr * ng + my_grp;
-      pos = (rr * nch + cc) * ng + my_grp;
-      last = cc == nch - 1;
-      if (++cc == nch) {
-        cc = 0;
-        ++rr;
-      }
-    } else {
-      const int i = j - own_full;
-      c = ucb + i;
-      tl = sc.R * ng + my_grp / sc.s;
-      pos = sc.R * ng * nch + (i < lmin ? i * sc.units + my_grp : lmin * sc.units + rank);
-      last = i == own_rem - 1;
-    }
+  EngOwnStages own(sc, my_grp);
+  int rot = 0, done = 0;
+  int pos, tl, c;
+  bool last;
+  while (own.next(pos, tl, c, last)) {
     // advance the ring position to stage `pos`
     slot += pos - done;
     done = pos + 1;
@@ -767,8 +671,8 @@ __device__ __forceinline__ bool eng_phase_products(const EngArgs& a, const EngPh
     }
   }
   // past the phase's last stage
-  slot += sc.R * ng * nch + rem_len_total - done;
-  seq += sc.R * ng * nch + rem_len_total;
+  slot += sc.total() - done;
+  seq += sc.total();
   while (slot >= a.n_slots) {
     slot -= a.n_slots;
     par ^= 1u;
