@@ -87,6 +87,25 @@ size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K);
 bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* packed,
                               bitnet_stream s);
 
+/* The same packing for weights that are already ternary x scale, with the scale taken the
+ * BitNet way: beta = |w| of the first non-zero weight in row-major order (1e-5 if all are
+ * zero, when every code is the zero weight anyway), then s_w, codes and trailer as above;
+ * exactly ternary x scale inputs get their ternary values back as codes.
+ * [I2S] "Known gaps": quantize_i2_s keeps the BitNet convention (scale = first non-zero
+ * |w|), so inputs must already be ternary x scale.  Errors as bitnet_pack_i2s. */
+bitnet_status bitnet_pack_i2s_prescaled(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                        bitnet_stream s);
+
+/* Validate an I2_S tensor of N x K weights (N*K/4 code bytes + 32-byte trailer) on the
+ * device.  counts: DEVICE int64[3], 8-byte aligned, overwritten asynchronously with
+ *   counts[0]  2-bit fields holding 3 (no ternary weight maps to it),
+ *   counts[1]  non-zero bytes among the 28 trailer bytes after the scale,
+ *   counts[2]  1 if the stored fp32 scale is not finite and positive, else 0.
+ * A tensor written by bitnet_pack_i2s(_prescaled) gives {0, 0, 0}.
+ * [I2S] "llama-quantize I2_S emits the canonical layout": ggml_validate_row_data accepts
+ * I2_S.  Errors: NULL, SHAPE (as bitnet_pack_i2s), ALIGN (packed 16 bytes, counts 8). */
+bitnet_status bitnet_validate_i2s(const uint8_t* packed, int64_t N, int64_t K, int64_t* counts, bitnet_stream s);
+
 /* BitNetRMSNorm + per-token absmax int8 quantisation of x [T, K] (bf16 or fp32).
  *   with gain:  ms = mean(x^2) (exact fixed-point sum, rounded once to fp32),
  *               inv = 1 / sqrt(ms + eps),  y = (x * inv) * gain      (fp32, no FMA)

@@ -150,6 +150,48 @@ def pack_i2s(W: np.ndarray) -> np.ndarray:
     return np.concatenate([body, trailer])
 
 
+def first_nonzero_scale(W: np.ndarray) -> np.float32:
+    """beta = |w| of the first non-zero weight in row-major order: the BitNet convention that
+    quantize_i2_s keeps for inputs that are already ternary x scale ("fix: I2_S ARM kernel
+    layout + squared-ReLU FFN", "Known gaps").  An all-zero tensor has no such weight; its
+    codes are all zero weights whatever the scale, and 1e-5 (the absmean floor) is stored."""
+    flat = np.asarray(W, dtype=F32).reshape(-1)
+    nz = np.flatnonzero(flat != 0)
+    return F32(abs(flat[nz[0]])) if nz.size else ABS_FLOOR
+
+
+def pack_i2s_prescaled(W: np.ndarray) -> np.ndarray:
+    """Ternary x scale fp32 weights [N, K] -> I2_S bytes, with beta = first_nonzero_scale(W)
+    and the codes of ternary_codes (for exactly ternary x scale inputs, w * (1 / beta) rounds
+    to -1, 0 or 1, the ternary value itself)."""
+    W = np.asarray(W, dtype=F32)
+    N, K = W.shape
+    if K % QBLOCK != 0:
+        raise ValueError("I2_S needs rows divisible by 128")
+    beta = first_nonzero_scale(W)
+    body = interleave_i2s(ternary_codes(W, beta))
+    trailer = np.zeros(TRAILER_BYTES, dtype=np.uint8)
+    trailer[:4] = np.frombuffer(np.asarray([beta], dtype="<f4").tobytes(), dtype=np.uint8)
+    return np.concatenate([body, trailer])
+
+
+def validate_i2s(packed: np.ndarray, N: int, K: int) -> tuple[int, int, int]:
+    """Checks of an I2_S tensor, the row-data validation that llama.cpp's
+    ggml_validate_row_data gains for I2_S in the same pull request (bullet "llama-quantize
+    I2_S emits the canonical layout"): (2-bit fields holding 3, which no ternary weight
+    maps to; non-zero bytes among the 28 trailer bytes after the scale; 1 if the stored
+    scale is not a finite positive fp32, else 0)."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    nb = N * K // 4
+    body = packed[:nb]
+    bad_codes = int(sum(int(np.count_nonzero(((body >> (2 * g)) & 3) == 3)) for g in range(4)))
+    trailer = packed[nb:nb + TRAILER_BYTES]
+    bad_trailer = int(np.count_nonzero(trailer[4:]))
+    beta = np.frombuffer(trailer[:4].tobytes(), dtype="<f4")[0]
+    bad_scale = 0 if (np.isfinite(beta) and beta > 0) else 1
+    return bad_codes, bad_trailer, bad_scale
+
+
 def unpack_i2s(packed: np.ndarray, N: int, K: int) -> tuple[np.ndarray, np.float32]:
     """I2_S bytes -> (codes uint8 [N, K], beta)."""
     packed = np.asarray(packed, dtype=np.uint8)

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
     sig = {
         "bitnet_i2s_packed_bytes": (c_sz, [c_i64, c_i64]),
         "bitnet_pack_i2s": (c_i, [c_p, c_i64, c_i64, c_p, c_p]),
+        "bitnet_pack_i2s_prescaled": (c_i, [c_p, c_i64, c_i64, c_p, c_p]),
+        "bitnet_validate_i2s": (c_i, [c_p, c_i64, c_i64, c_p, c_p]),
         "bitnet_rmsnorm_quant_act": (c_i, [c_p, c_i, c_p, c_f, c_i64, c_i64, c_p, c_p, c_p, c_p]),
         "bitnet_bitlinear": (c_i, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i, c_p, c_p]),
         "bitnet_bitlinear_group": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_i64, c_i64, c_p, c_i, c_p]),
@@ -137,6 +139,29 @@ def pack_i2s(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> t
         out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     _check(lib().bitnet_pack_i2s(_ptr(W), N, K, _ptr(out), _stream(stream)), "pack_i2s")
     return out
+
+
+def pack_i2s_prescaled(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Ternary x scale fp32 weights [N, K] -> I2_S bytes, scale = first non-zero |w|."""
+    _need(W, "W")
+    N, K = W.shape
+    nbytes = i2s_packed_bytes(N, K)
+    if nbytes == 0:
+        raise BitnetError(2, "pack_i2s_prescaled")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check(lib().bitnet_pack_i2s_prescaled(_ptr(W), N, K, _ptr(out), _stream(stream)), "pack_i2s_prescaled")
+    return out
+
+
+def validate_i2s(packed: torch.Tensor, N: int, K: int, counts: torch.Tensor | None = None, stream=None):
+    """Device-side I2_S checks -> int64 [3] device tensor: (fields holding 3, non-zero
+    trailer bytes after the scale, 1 if the scale is not finite and positive)."""
+    _need(packed, "packed")
+    if counts is None:
+        counts = torch.empty(3, dtype=torch.int64, device=packed.device)
+    _check(lib().bitnet_validate_i2s(_ptr(packed), N, K, _ptr(counts), _stream(stream)), "validate_i2s")
+    return counts
 
 
 def rmsnorm_quant_act(x: torch.Tensor, gain: torch.Tensor | None, eps: float = 1e-6, out=None, stream=None):

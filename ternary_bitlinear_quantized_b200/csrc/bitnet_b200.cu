@@ -464,11 +464,11 @@ size_t bitnet_i2s_packed_bytes(int64_t N, int64_t K) {
   return (size_t)(N * K / 4 + 32);
 }
 
-bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* packed, bitnet_stream stream) {
+static bitnet_status enqueue_pack(const float* W, int64_t N, int64_t K, uint8_t* packed, int prescaled,
+                                  cudaStream_t s) {
   if (!W || !packed) return BITNET_ERR_NULL;
   if (N <= 0 || K <= 0 || K % 128 != 0 || N * K >= (1ll << 40)) return BITNET_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(packed)) return BITNET_ERR_ALIGN;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long n = N * K;
   PackScratch* sc = reinterpret_cast<PackScratch*>(packed + n / 4);
   const int sms = device_sm_count();
@@ -477,16 +477,52 @@ bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* pac
   long long wantc = (n / 16 + 255) / 256;
   const unsigned gridc = (unsigned)(wantc < sms * 16 ? wantc : sms * 16);
   cudaError_t e;
-  if ((e = launch(k_pack_clear, dim3(1), dim3(1), 0, s, false, sc)) != cudaSuccess) return cuda_fail(e, "k_pack_clear");
-  if ((e = launch(k_pack_absmax, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
-    return cuda_fail(e, "k_pack_absmax");
-  if ((e = launch(k_pack_sum, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
-    return cuda_fail(e, "k_pack_sum");
+  if (prescaled) {
+    if ((e = launch(k_pack_first_nz_clear, dim3(1), dim3(1), 0, s, false, sc)) != cudaSuccess)
+      return cuda_fail(e, "k_pack_first_nz_clear");
+    if ((e = launch(k_pack_first_nz, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
+      return cuda_fail(e, "k_pack_first_nz");
+  } else {
+    if ((e = launch(k_pack_clear, dim3(1), dim3(1), 0, s, false, sc)) != cudaSuccess) return cuda_fail(e, "k_pack_clear");
+    if ((e = launch(k_pack_absmax, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
+      return cuda_fail(e, "k_pack_absmax");
+    if ((e = launch(k_pack_sum, dim3(grid), dim3(256), 0, s, false, W, n, sc)) != cudaSuccess)
+      return cuda_fail(e, "k_pack_sum");
+  }
   if ((e = launch(k_pack_codes, dim3(gridc), dim3(256), 0, s, false, W, n, (const PackScratch*)sc,
-                  reinterpret_cast<uint32_t*>(packed))) != cudaSuccess)
+                  reinterpret_cast<uint32_t*>(packed), prescaled)) != cudaSuccess)
     return cuda_fail(e, "k_pack_codes");
-  if ((e = launch(k_pack_trailer, dim3(1), dim3(1), 0, s, false, sc, n)) != cudaSuccess)
+  if ((e = launch(k_pack_trailer, dim3(1), dim3(1), 0, s, false, sc, n, W, prescaled)) != cudaSuccess)
     return cuda_fail(e, "k_pack_trailer");
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_pack_i2s(const float* W, int64_t N, int64_t K, uint8_t* packed, bitnet_stream stream) {
+  return enqueue_pack(W, N, K, packed, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_pack_i2s_prescaled(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                        bitnet_stream stream) {
+  return enqueue_pack(W, N, K, packed, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_validate_i2s(const uint8_t* packed, int64_t N, int64_t K, int64_t* counts,
+                                  bitnet_stream stream) {
+  if (!packed || !counts) return BITNET_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % 128 != 0 || N * K >= (1ll << 40)) return BITNET_ERR_SHAPE;
+  if (!aligned16(packed) || (reinterpret_cast<uintptr_t>(counts) & 7)) return BITNET_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long nwords = N * K / 16;
+  const int sms = device_sm_count();
+  const long long want = (nwords + 255) / 256;
+  const unsigned grid = (unsigned)(want < sms * 8 ? want : sms * 8);
+  unsigned long long* c = reinterpret_cast<unsigned long long*>(counts);
+  cudaError_t e;
+  if ((e = launch(k_validate_clear, dim3(1), dim3(1), 0, s, false, c)) != cudaSuccess)
+    return cuda_fail(e, "k_validate_clear");
+  if ((e = launch(k_validate_i2s, dim3(grid), dim3(256), 0, s, false, reinterpret_cast<const uint32_t*>(packed), nwords,
+                  packed + N * K / 4, c)) != cudaSuccess)
+    return cuda_fail(e, "k_validate_i2s");
   return BITNET_OK;
 }
 

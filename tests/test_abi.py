@@ -65,6 +65,14 @@ def test_argument_checks_before_launch(L):
     assert L.bitnet_ffn_block(p, 0, None, p, p, None, p, 1, 256, 384, 0, 1e-6, p, 0, p, 16, None) == 5
     assert L.bitnet_ffn_block(p, 0, None, p, p, None, p, 1, 256, 300, 0, 1e-6, p, 0, p, 1 << 20, None) == 2
     assert L.bitnet_ffn_block(p, 0, None, p, p, None, p, 1, 256, 384, 5, 1e-6, p, 0, p, 1 << 20, None) == 4
+    assert L.bitnet_pack_i2s_prescaled(None, 4, 128, p, None) == 1
+    assert L.bitnet_pack_i2s_prescaled(p, 4, 200, p, None) == 2
+    assert L.bitnet_pack_i2s_prescaled(p, 4, 128, odd, None) == 3
+    assert L.bitnet_validate_i2s(None, 4, 128, p, None) == 1
+    assert L.bitnet_validate_i2s(p, 4, 128, None, None) == 1
+    assert L.bitnet_validate_i2s(p, 0, 128, p, None) == 2
+    assert L.bitnet_validate_i2s(odd, 4, 128, p, None) == 3
+    assert L.bitnet_validate_i2s(p, 4, 128, ctypes.c_void_p(20), None) == 3  # counts must be 8-byte aligned
 
 
 def test_status_strings(L):

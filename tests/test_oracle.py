@@ -412,3 +412,58 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
         check = lambda: test_ffn_block_matches_textbook("relu2")
     with pytest.raises(AssertionError):
         check()
+
+
+# ----------------------------------------------------------------------------- prescaled pack, validator
+
+def _ternary_times_scale(N, K, scale, seed, density=0.7):
+    rng = np.random.default_rng(seed)
+    t = rng.choice(np.array([-1, 0, 1], dtype=np.int8), size=(N, K), p=[density / 2, 1 - density, density / 2])
+    return t, (t.astype(F32) * F32(scale))
+
+
+def test_prescaled_pack_recovers_scale_and_ternary_values():
+    """quantize_i2_s's convention: inputs are ternary x scale and the scale is the first
+    non-zero |w|; so the stored scale is that scale exactly and the codes are t + 1."""
+    t, W = _ternary_times_scale(3, 256, 0.0374, 1)
+    p = O.pack_i2s_prescaled(W)
+    codes, beta = O.unpack_i2s(p, 3, 256)
+    assert beta == F32(0.0374)
+    assert np.array_equal(codes.astype(np.int16) - 1, t)
+    # the same code bytes as the absmean pack (whose scale is smaller: scale x density)
+    pa = O.pack_i2s(W)
+    assert np.array_equal(p[:3 * 256 // 4], pa[:3 * 256 // 4])
+    assert O.unpack_i2s(pa, 3, 256)[1] < beta
+
+
+def test_prescaled_pack_first_nonzero_in_row_major_order():
+    W = np.zeros((2, 128), dtype=F32)
+    W[1, 5] = F32(0.25)      # later in row-major order
+    W[0, 100] = F32(-0.7)    # first non-zero: row 0 comes first
+    W[0, 120] = F32(0.7)
+    p = O.pack_i2s_prescaled(W)
+    codes, beta = O.unpack_i2s(p, 2, 128)
+    assert beta == F32(0.7)
+    assert codes[0, 100] == 0 and codes[0, 120] == 2 and codes[1, 5] == 1  # 0.25 / 0.7 rounds to 0
+    z = O.pack_i2s_prescaled(np.zeros((1, 128), dtype=F32))
+    zc, zb = O.unpack_i2s(z, 1, 128)
+    assert zb == F32(1e-5) and np.all(zc == 1)
+
+
+def test_validate_i2s_counts_planted_faults():
+    W = workloads.latent_weight(4, 256, 3, "validate").numpy()
+    p = O.pack_i2s(W)
+    assert O.validate_i2s(p, 4, 256) == (0, 0, 0)
+    bad = p.copy()
+    bad[5] |= 0b11000000           # field 0 of byte 5 -> 3
+    bad[77] |= 0b00001111          # fields 2 and 3 of byte 77 -> 3
+    assert O.validate_i2s(bad, 4, 256) == (3, 0, 0)
+    nb = 4 * 256 // 4
+    tr = p.copy()
+    tr[nb + 10] = 7                # a trailer byte after the scale
+    tr[nb + 31] = 1
+    assert O.validate_i2s(tr, 4, 256) == (0, 2, 0)
+    for val in (np.nan, np.inf, -1.0, 0.0):
+        sc = p.copy()
+        sc[nb:nb + 4] = np.frombuffer(np.asarray([val], dtype="<f4").tobytes(), dtype=np.uint8)
+        assert O.validate_i2s(sc, 4, 256) == (0, 0, 1), val

@@ -65,6 +65,46 @@ def test_pack_repeatable_across_streams():
 
 # ----------------------------------------------------------------------------- a2: quant
 
+@pytest.mark.parametrize("N,K,case", [(1, 128, "ternary"), (17, 384, "ternary"), (300, 640, "ternary"),
+                                      (64, 6912, "ternary"), (33, 256, "latent"), (5, 128, "leading_zeros"),
+                                      (3, 256, "zeros")])
+def test_pack_prescaled_bytes_bitexact(N, K, case):
+    """Prescaled packing (scale = first non-zero |w|) against the oracle, byte for byte."""
+    rng = np.random.default_rng(N * 7 + K)
+    if case == "ternary":
+        t = rng.choice(np.array([-1, 0, 1], dtype=np.int8), size=(N, K), p=[0.35, 0.3, 0.35])
+        W = t.astype(np.float32) * np.float32(0.0213 * (1 + N % 5))
+    elif case == "latent":
+        W = workloads.latent_weight(N, K, 5, "prescaled").numpy()
+    elif case == "leading_zeros":
+        W = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+        W.reshape(-1)[: N * K // 2 + 3] = 0.0
+    else:
+        W = np.zeros((N, K), dtype=np.float32)
+    got = tb.pack_i2s_prescaled(torch.from_numpy(W).to(DEV)).cpu().numpy()
+    ref = O.pack_i2s_prescaled(W)
+    assert np.array_equal(got, ref)
+    if case == "ternary":
+        codes, beta = O.unpack_i2s(got, N, K)
+        assert np.array_equal(codes.astype(np.int16) - 1, t)
+
+
+@pytest.mark.parametrize("N,K", [(4, 256), (300, 640), (2560, 2560)])
+def test_validate_i2s_matches_oracle(N, K):
+    W = workloads.latent_weight(N, K, 11, "validate")
+    p = gpu_pack(W)
+    assert tuple(tb.validate_i2s(p, N, K).cpu().tolist()) == (0, 0, 0)
+    bad = p.cpu().numpy().copy()
+    rng = np.random.default_rng(N + K)
+    nb = N * K // 4
+    idx = rng.choice(nb, size=min(50, nb), replace=False)
+    bad[idx] |= 0b00110000                      # field 1 of those bytes -> 3
+    bad[nb + 9] = 1                             # a trailer byte after the scale
+    bad[nb:nb + 4] = np.frombuffer(np.asarray([np.nan], dtype="<f4").tobytes(), dtype=np.uint8)
+    got = tuple(tb.validate_i2s(torch.from_numpy(bad).to(DEV), N, K).cpu().tolist())
+    assert got == O.validate_i2s(bad, N, K) == (len(idx), 1, 1)
+
+
 @pytest.mark.parametrize("T,K,dtype,use_gain,outliers", [
     (1, 2560, torch.bfloat16, True, False),
     (5, 640, torch.bfloat16, True, True),
