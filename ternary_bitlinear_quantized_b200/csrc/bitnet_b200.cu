@@ -128,10 +128,11 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
                                    int8_t* q, float* s_x, int32_t* sum_q, cudaStream_t s) {
   if (T == 0) return BITNET_OK;
   // Rows of up to 8192 values (K a multiple of 8, 16-byte aligned rows): values in registers,
-  // one to four warps per row.
+  // one to four warps per row; four when there are too few rows to fill the GPU, so each
+  // row's reductions are short.
   const size_t esz_r = xt == BITNET_BF16 ? 2 : 4;
   if (K <= 4 * 2048 && K % 8 == 0 && aligned16(x) && aligned16(q) && (K * esz_r) % 16 == 0) {
-    const int w = K <= 2048 ? 1 : (K <= 4096 ? 2 : 4);
+    const int w = (T <= 256 || K > 4096) ? 4 : (K <= 2048 ? 1 : 2);
     const unsigned grid = (unsigned)((T + QW_THREADS / 32 / w - 1) / (QW_THREADS / 32 / w));
     cudaError_t e;
     if (xt == BITNET_BF16) {
@@ -364,9 +365,11 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
     const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
     const int per = (p.n_tiles + grid - 1) / grid * NT * GEMV_ROWS * a.T;
     if (per > acc_ints) acc_ints = per;
-    // Activations staged in shared memory: always for SRC_LOCAL, else when they fit.
+    // Activations staged in shared memory: always for SRC_LOCAL; given ones when they fit
+    // and a CTA has at least three tiles to reuse them over (else the copy is only latency).
     const int xp = (p.K + 255) / 256 * 256 + 64;
-    if ((p.src == SRC_LOCAL || a.T * xp <= ENG_QS_GLOBAL_MAX) && a.T * xp > qs) qs = a.T * xp;
+    a.ph[i].xstage = p.src == SRC_GLOBAL && a.T * xp <= ENG_QS_GLOBAL_MAX && (p.n_tiles + grid - 1) / grid >= 3;
+    if ((p.src == SRC_LOCAL || a.ph[i].xstage) && a.T * xp > qs) qs = a.T * xp;
   }
   qs = (qs + 127) / 128 * 128;
   acc_ints = (acc_ints + 3) / 4 * 4;

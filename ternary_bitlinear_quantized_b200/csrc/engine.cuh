@@ -81,6 +81,7 @@ struct EngPhase {
   float* pmax;
   long long* psum;
   int bar_a, bar_b;
+  int xstage;  // SRC_GLOBAL: copy the activations into shared memory first (else read in place)
   // Stage geometry: a stage is one 2-D TMA box per tensor of 16 rows (one tile) x
   // chunk_words 32-bit words (a K-chunk; chunk_words = 16 mod 32, so the rows of a box are
   // 64 mod 128 bytes apart); stage_bytes = tensors x 64 x chunk_words.
@@ -841,7 +842,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
       // Activations of this phase: in shared memory (layout eng_perm) when they fit, else
       // read in plain order from global memory.
       const bool local = p.src == SRC_LOCAL;
-      const bool xsm = local || T * xp <= a.qs_bytes;
+      const bool xsm = local || p.xstage;
       if (local) {
         for (int t = 0; t < T; ++t) {
           quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
