@@ -244,6 +244,15 @@ bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_d
  * the last read. */
 bitnet_status bitnet_get_device_status(bitnet_stream s);
 
+/* Test and debugging aid (no counterpart on the pages): sets the limit of every bounded wait
+ * in the kernels on the CURRENT device, in SM clock cycles (<= 0 restores the default of
+ * 2e9, about a second).  A wait that runs past the limit gives up, sets BITNET_ERR_TIMEOUT in
+ * the device status word and the kernel returns early with its outputs incomplete (it still
+ * lets its own in-flight copies land, with a fixed limit).  Tests use a short limit to make
+ * waits run out on purpose.  Synchronises the device before and after; call it only while no
+ * kernel of this library runs.  Errors: CUDA. */
+bitnet_status bitnet_debug_set_wait_limit(long long cycles);
+
 /* Static English text of a status code. */
 const char* bitnet_status_string(bitnet_status st);
 

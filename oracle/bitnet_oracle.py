@@ -28,7 +28,7 @@ What each function follows (pages by title):
   as named by both pages above and by "More BitNet-like IQ1_S quantizations"
   (llama.cpp discussion: 8-bit activations, ternary weights).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * bit order inside an I2_S block: element 128 b + 32 g + i is byte 32 b + i, bits
   (7 - 2g):(6 - 2g) -- the interleaved layout, as opposed to the "sequential (byte

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
                                        c_i64, c_i64, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_p, c_p, c_p, c_p, c_i,
                                        c_p, c_sz, c_p]),
         "bitnet_get_device_status": (c_i, [c_p]),
+        "bitnet_debug_set_wait_limit": (c_i, [ctypes.c_longlong]),
         "bitnet_status_string": (ctypes.c_char_p, [c_i]),
         "bitnet_last_error": (ctypes.c_char_p, []),
     }
@@ -288,6 +289,12 @@ def decoder_block(x, attn_out, gains: dict, packed: dict, NKV: int, I: int, act:
                                       _ptr(outs["ffn"]), _dtype_code(outs["ffn"].dtype), _ptr(ws), ws.numel(),
                                       _stream(stream)), "decoder_block")
     return outs
+
+
+def debug_set_wait_limit(cycles: int) -> None:
+    """Set the kernels' bounded-wait limit on the current device (cycles; <= 0 restores the
+    default).  A testing aid: synchronises the device."""
+    _check(lib().bitnet_debug_set_wait_limit(int(cycles)), "debug_set_wait_limit")
 
 
 def device_status(stream=None) -> int:

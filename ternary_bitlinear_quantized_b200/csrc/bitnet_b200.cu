@@ -2,6 +2,7 @@
 // order of launches on the caller's stream.  Every step of the arithmetic runs in the
 // kernels of quant.cuh, pack.cuh, engine.cuh and gemm_tc.cuh (one translation unit, so
 // that the device status word needs no relocatable device code).
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -61,20 +62,22 @@ static int device_sm_count() {
   return cached_sms > 0 ? cached_sms : 148;
 }
 
-// Opt a kernel in to the full dynamic shared memory of the SM, once per device.
+// Opt a kernel in to the full dynamic shared memory of the SM, once per device.  The
+// "done" flags are atomics: several host threads may race to set the same attribute, which
+// is harmless (the same value), and none of them reads a torn flag.
 static cudaError_t opt_in_smem(const void* kern, int slot) {
-  static int done[8][64] = {};
+  static std::atomic<int> done[16][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  int& d = done[slot & 7][dev & 63];
-  if (d) return cudaSuccess;
+  std::atomic<int>& d = done[slot & 15][dev & 63];
+  if (d.load(std::memory_order_acquire)) return cudaSuccess;
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin - (int)fa.sharedSizeBytes);
-  if (e == cudaSuccess) d = 1;
+  if (e == cudaSuccess) d.store(1, std::memory_order_release);
   return e;
 }
 
@@ -83,15 +86,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a function-local static is initialised
+// exactly once even when several threads call this at the same time).
 static EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -157,17 +162,17 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
   cudaError_t e;
   if (smem > 48 * 1024) {
     // Opt in to the large dynamic shared memory once per device and kernel.
-    static int done_mask[2][64] = {};
+    static std::atomic<int> done_mask[2][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    int& done = done_mask[xt == BITNET_BF16 ? 0 : 1][dev & 63];
-    if (!done) {
+    std::atomic<int>& done = done_mask[xt == BITNET_BF16 ? 0 : 1][dev & 63];
+    if (!done.load(std::memory_order_acquire)) {
       e = xt == BITNET_BF16 ? cudaFuncSetAttribute(k_rmsnorm_quant<__nv_bfloat16>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, BITNET_MAX_K * 4)
                             : cudaFuncSetAttribute(k_rmsnorm_quant<float>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, BITNET_MAX_K * 4);
       if (e != cudaSuccess) return cuda_fail(e, "quant attribute");
-      done = 1;
+      done.store(1, std::memory_order_release);
     }
   }
   if (xt == BITNET_BF16) {
@@ -724,10 +729,10 @@ static bitnet_status enqueue_ffn_launches(const void* x, bitnet_dtype xt, const 
   return enqueue_gemv(q_h, s_h, sum_h, 1, pd, nH, o, nullptr, T, I, ot, false, act, nullptr, s);
 }
 
-bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
-                               const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T, int64_t H,
-                               int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot, void* ws,
-                               size_t ws_bytes, bitnet_stream stream) {
+// Checks of bitnet_ffn_block's arguments other than the workspace (BITNET_OK also for T = 0).
+static bitnet_status ffn_check_args(const void* x, bitnet_dtype xt, const uint8_t* p_gate, const uint8_t* p_up,
+                                    const uint8_t* p_down, int64_t T, int64_t H, int64_t I, bitnet_act act,
+                                    const void* out, bitnet_dtype ot, const float* g_ffn, const float* g_sub) {
   if (xt != BITNET_BF16 && xt != BITNET_F32) return BITNET_ERR_DTYPE;
   if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
   if (act != BITNET_RELU2 && act != BITNET_SILU) return BITNET_ERR_DTYPE;
@@ -735,11 +740,21 @@ bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ff
     return BITNET_ERR_SHAPE;
   if (T == 0) return BITNET_OK;
   if (!x || !p_gate || !p_up || !p_down || !out) return BITNET_ERR_NULL;
+  if (!aligned16(x) || !aligned16(p_gate) || !aligned16(p_up) || !aligned16(p_down) || !aligned16(out) ||
+      (g_ffn && !aligned16(g_ffn)) || (g_sub && !aligned16(g_sub)))
+    return BITNET_ERR_ALIGN;
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_ffn_block(const void* x, bitnet_dtype xt, const float* g_ffn, const uint8_t* p_gate,
+                               const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T, int64_t H,
+                               int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot, void* ws,
+                               size_t ws_bytes, bitnet_stream stream) {
+  bitnet_status st0 = ffn_check_args(x, xt, p_gate, p_up, p_down, T, H, I, act, out, ot, g_ffn, g_sub);
+  if (st0 != BITNET_OK || T == 0) return st0;
   if (!ws) return BITNET_ERR_WORKSPACE;
   if (ws_bytes < bitnet_ffn_workspace_bytes(T, H, I)) return BITNET_ERR_WORKSPACE;
-  if (!aligned16(x) || !aligned16(p_gate) || !aligned16(p_up) || !aligned16(p_down) || !aligned16(out) ||
-      !aligned16(ws) || (g_ffn && !aligned16(g_ffn)) || (g_sub && !aligned16(g_sub)))
-    return BITNET_ERR_ALIGN;
+  if (!aligned16(ws)) return BITNET_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   if (T > ENG_MAX_T || !eng_quant_ok(H) || !eng_quant_ok(I))
@@ -792,8 +807,10 @@ bitnet_status bitnet_ffn_block_noalloc(const void* x, bitnet_dtype xt, const flo
                                        const uint8_t* p_up, const float* g_sub, const uint8_t* p_down, int64_t T,
                                        int64_t H, int64_t I, bitnet_act act, float eps, void* out, bitnet_dtype ot,
                                        bitnet_stream stream) {
-  if (T < 0 || H <= 0 || I <= 0) return BITNET_ERR_SHAPE;
-  if (T == 0) return BITNET_OK;
+  // The same argument checks as bitnet_ffn_block, all before the shared scratch is touched,
+  // so that an invalid call writes nothing and returns the same status.
+  bitnet_status st = ffn_check_args(x, xt, p_gate, p_up, p_down, T, H, I, act, out, ot, g_ffn, g_sub);
+  if (st != BITNET_OK || T == 0) return st;
   const size_t need = bitnet_ffn_workspace_bytes(T, H, I);
   if (need == 0) return BITNET_ERR_SHAPE;
   if (need > kNoAllocScratchBytes) {
@@ -802,7 +819,7 @@ bitnet_status bitnet_ffn_block_noalloc(const void* x, bitnet_dtype xt, const flo
     return BITNET_ERR_WORKSPACE;
   }
   uint8_t* ws = nullptr;
-  bitnet_status st = noalloc_scratch(&ws);
+  st = noalloc_scratch(&ws);
   if (st != BITNET_OK) return st;
   // The grid-barrier counters must start at zero; the previous call normally leaves them
   // zero, but clear them anyway (a call that timed out would not have).
@@ -928,6 +945,14 @@ bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_d
   plan_ffn(ea, bar, po.arrive_barrier, out_o, ot == BITNET_F32, g_ffn_norm, p_gate, p_up, g_ffn_sub_norm, p_down, T,
            H, I, act, out_ffn, ot, wf);
   return enqueue_engine(ea, s);
+}
+
+bitnet_status bitnet_debug_set_wait_limit(long long cycles) {
+  if (cycles <= 0) cycles = kDefaultWaitLimitCycles;
+  BN_CUDA(cudaDeviceSynchronize(), "wait limit (synchronize)");
+  BN_CUDA(cudaMemcpyToSymbol(c_wait_limit, &cycles, sizeof(cycles)), "wait limit (copy)");
+  BN_CUDA(cudaDeviceSynchronize(), "wait limit (synchronize)");
+  return BITNET_OK;
 }
 
 bitnet_status bitnet_get_device_status(bitnet_stream stream) {

@@ -82,19 +82,37 @@ BN_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of a barrier, giving up after about a second of clock
-// cycles: then the device status word is set to BITNET_ERR_TIMEOUT and false returned.
-constexpr long long kWaitLimitCycles = 2000000000ll;
+// Limit of every bounded wait, in SM clock cycles (about a second by default).  A wait that
+// runs past it gives up: the device status word is set to BITNET_ERR_TIMEOUT and the kernel
+// leaves its loops.  bitnet_debug_set_wait_limit() changes it between launches (tests use a
+// short limit to make waits run out on purpose).
+constexpr long long kDefaultWaitLimitCycles = 2000000000ll;
+__constant__ long long c_wait_limit = kDefaultWaitLimitCycles;
+// After a wait has given up, the copies a CTA issued into its own shared memory are still
+// awaited before it exits, with this fixed limit (not the settable one): they are plain reads
+// of global memory and always land.
+constexpr long long kDrainLimitCycles = 2000000000ll;
+
+// Wait for phase `parity` of a barrier, giving up after c_wait_limit clock cycles: then the
+// device status word is set to BITNET_ERR_TIMEOUT and false returned.
 BN_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  const long long t0 = clock64(), lim = c_wait_limit;
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > lim) {
       atomicExch(&g_device_status, (int)BITNET_ERR_TIMEOUT);
       return false;
     }
   }
   return true;
+}
+
+// Wait, with the fixed drain limit, for phase `parity` of a barrier that a copy into this
+// CTA's shared memory completes (used on the way out after another wait gave up).
+BN_DEV void mbar_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 <= kDrainLimitCycles) {
+  }
 }
 
 // Bulk copy global -> this CTA's shared memory, completing `bytes` on barrier `bar`

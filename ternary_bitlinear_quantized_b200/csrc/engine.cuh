@@ -377,7 +377,7 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
       if (v >= target) break;
       const long long now = clock64();
       if (t0 < 0) t0 = now;
-      if (now - t0 > kWaitLimitCycles) {
+      if (now - t0 > c_wait_limit) {
         atomicExch(&g_device_status, (int)BITNET_ERR_TIMEOUT);
         ok = false;
         break;
@@ -539,9 +539,9 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
 // barrier waits).
 BN_DEV bool wait_slot_tag(const volatile int* tag, int want) {
   if (*tag == want) return true;
-  const long long t0 = clock64();
+  const long long t0 = clock64(), lim = c_wait_limit;
   while (*tag != want) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > lim) {
       atomicExch(&g_device_status, (int)BITNET_ERR_TIMEOUT);
       return false;
     }

@@ -75,6 +75,31 @@ def test_argument_checks_before_launch(L):
     assert L.bitnet_validate_i2s(p, 4, 128, ctypes.c_void_p(20), None) == 3  # counts must be 8-byte aligned
 
 
+def test_noalloc_checks_arguments_like_ffn_block(L):
+    """The no-alloc FFN entry answers invalid arguments with the same status as
+    bitnet_ffn_block, before it touches its built-in scratch (no CUDA call is made)."""
+    p = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(17)
+    big = 1 << 30
+    cases = [  # (x, xt, p_gate, T, H, I, act, out, ot)
+        (p, 7, p, 1, 256, 384, 0, p, 0),        # bad x dtype
+        (p, 0, p, 1, 256, 384, 0, p, 9),        # bad out dtype
+        (p, 0, p, 1, 256, 384, 5, p, 0),        # bad activation
+        (p, 0, p, 1, 200, 384, 0, p, 0),        # H % 128
+        (p, 0, p, 1, 256, 300, 0, p, 0),        # I % 128
+        (p, 0, p, 1, 1 << 20, 384, 0, p, 0),    # H beyond the maximum
+        (p, 0, p, -1, 256, 384, 0, p, 0),       # negative T
+        (None, 0, p, 1, 256, 384, 0, p, 0),     # NULL input
+        (p, 0, None, 1, 256, 384, 0, p, 0),     # NULL weights
+        (odd, 0, p, 1, 256, 384, 0, p, 0),      # misaligned input
+    ]
+    for x, xt, pg, T, H, I, act, out, ot in cases:
+        want = L.bitnet_ffn_block(x, xt, None, pg, p, None, p, T, H, I, act, 1e-6, out, ot, p, big, None)
+        got = L.bitnet_ffn_block_noalloc(x, xt, None, pg, p, None, p, T, H, I, act, 1e-6, out, ot, None)
+        assert want != 0 and got == want, (T, H, I, want, got)
+    assert L.bitnet_ffn_block_noalloc(p, 0, None, p, p, None, p, 0, 256, 384, 0, 1e-6, p, 0, None) == 0  # T = 0
+
+
 def test_status_strings(L):
     for code in range(8):
         assert L.bitnet_status_string(code)

@@ -18,6 +18,7 @@ import torch
 
 from oracle import bitnet_oracle as O
 import workloads
+from tests.tie_inputs import tie_activations, tie_weights
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 F32 = np.float32
@@ -230,6 +231,26 @@ def test_quant_ties_round_half_even():
     assert list(q[0, 1:1 + len(halves)]) == [0, 2, 2, 4, 0, -2, -2, 100]
 
 
+def test_ties_of_codes_and_activations_round_half_even():
+    """The tie fixtures land on exact .5 ties and round half to even: weights +-0.5 beta -> 0,
+    +-1.5 beta -> +-1 (after the clamp); activations (n + 1/2)/64 with s_x = 64 -> the even
+    neighbour."""
+    W = tie_weights()
+    assert O.absmean_scale(W) == F32(2.0 ** -6)
+    codes, _ = O.unpack_i2s(O.pack_i2s(W), *W.shape)
+    want = np.where(np.abs(W) < 2.0 ** -6, 0, np.sign(W)).astype(np.int16)
+    assert np.array_equal(codes.astype(np.int16) - 1, want)
+    x = tie_activations()
+    q, s, _ = O.rmsnorm_quant_act(x, None, 1e-6)
+    assert np.all(s == F32(64.0))
+    for t in range(x.shape[0]):
+        for k in range(x.shape[1]):
+            v = Fraction(float(x[t, k])) * 64
+            lo = math.floor(v)
+            want_q = lo if (v - lo != Fraction(1, 2) or lo % 2 == 0) else lo + 1
+            assert q[t, k] == max(-128, min(127, want_q))
+
+
 def test_rmsnorm_matches_textbook():
     x = bf16_inputs(4, 2560, 5)
     g = workloads.gain(2560, 0, "pin").numpy()
@@ -360,6 +381,86 @@ def test_ffn_block_matches_textbook(act):
     assert np.linalg.norm(out - ref) / np.linalg.norm(ref) <= 2e-3
 
 
+def textbook_block(x, attn_out, gains, W, act, eps=1e-6):
+    """The decoder block's projections in fp64 from the plain formulas: q, k, v from x
+    through attn_norm; o from the attention output through attn_sub_norm; the FFN (its own
+    textbook) from o's output through ffn_norm and ffn_sub_norm."""
+    def norm_quant(v, gain):
+        v = v.astype(np.float64)
+        y = v / np.sqrt(np.mean(v * v, axis=1, keepdims=True) + eps) * gain.astype(np.float64)
+        s = 127.0 / np.maximum(np.max(np.abs(y), axis=1, keepdims=True), 1e-5)
+        return np.clip(np.round(y * s), -128, 127) / s
+
+    def ternary(Wm):
+        Wm = Wm.astype(np.float64)
+        beta = max(np.mean(np.abs(Wm)), 1e-5)
+        return np.clip(np.round(Wm / beta), -1, 1) * beta
+
+    xq = norm_quant(x, gains["attn_norm"])
+    out = {nm: xq @ ternary(W[nm]).T for nm in ("q", "k", "v")}
+    out["o"] = norm_quant(attn_out, gains["attn_sub_norm"]) @ ternary(W["o"]).T
+    out["ffn"] = textbook_ffn(out["o"], gains["ffn_norm"], W["gate"], W["up"], gains["ffn_sub_norm"], W["down"], act,
+                              eps)
+    return out
+
+
+def _tiny_block(seed=3, T=2):
+    # n_q == hidden, so attn_norm and attn_sub_norm have the same length and a swap of the
+    # two would not fail on shapes alone.
+    sh = workloads.BlockShape("tiny", hidden=256, n_q=256, n_kv=128, inter=384, act="relu2")
+    d = workloads.block_inputs(sh, T=T, seed=seed)
+    W = {nm: d["W_" + nm].numpy() for nm in sh.tensors()}
+    packed = {nm: O.pack_i2s(W[nm]) for nm in sh.tensors()}
+    gains = {k[2:]: v.numpy() for k, v in d.items() if k.startswith("g_")}
+    xb = O.bf16_bits_to_f32(d["x"].view(torch.int16).numpy().view(np.uint16))
+    ab = O.bf16_bits_to_f32(d["attn_out"].view(torch.int16).numpy().view(np.uint16))
+    return sh, W, packed, gains, xb, ab
+
+
+def test_decoder_block_matches_textbook(block_fn=None):
+    """Each projection of the oracle's block against an fp64 textbook computation that takes
+    its own gain and its own input ("Add optional RMSNorm support to BitNet quantization": a
+    BitLinear normalises its own input; the per-block norms attn_norm, attn_sub_norm,
+    ffn_norm, ffn_sub_norm of "More BitNet-like IQ1_S quantizations")."""
+    block_fn = block_fn or O.decoder_block
+    sh, W, packed, gains, xb, ab = _tiny_block()
+    out = block_fn(xb, ab, gains, packed, sh.tensors(), "relu2", 1e-6, "f32")
+    ref = textbook_block(xb, ab, gains, W, "relu2")
+    for nm in ("q", "k", "v", "o", "ffn"):
+        err = np.linalg.norm(out[nm] - ref[nm]) / np.linalg.norm(ref[nm])
+        assert err <= 2e-3, f"{nm}: relative error {err}"
+
+
+def _block_mutant(kind):
+    """A copy of the oracle's decoder_block with one plausible routing mistake."""
+    def block(x, attn_out, gains, packed, shape, act, eps, out_dtype="bf16"):
+        g = dict(gains)
+        if kind == "norms_swapped":
+            g["attn_norm"], g["attn_sub_norm"] = gains["attn_sub_norm"], gains["attn_norm"]
+        qkv_in = attn_out if kind == "qkv_from_attn_out" else x
+        out = {}
+        q, s, sq = O.rmsnorm_quant_act(qkv_in, g["attn_norm"], eps)
+        for nm in ("q", "k", "v"):
+            N, K = shape[nm]
+            out[nm] = O.bitlinear(q, s, sq, packed[nm], N, K, out_dtype)
+        N, K = shape["o"]
+        out["o"] = O.bitlinear_from_x(attn_out, g["attn_sub_norm"], eps, packed["o"], N, K, out_dtype)
+        I, H = shape["gate"]
+        ffn_in = x if kind == "ffn_from_block_input" else out["o"]
+        ffn_norm = g["ffn_sub_norm"][:H] if kind == "ffn_norms_swapped" else g["ffn_norm"]
+        out["ffn"] = O.ffn_block(ffn_in, ffn_norm, packed["gate"], packed["up"], g["ffn_sub_norm"], packed["down"],
+                                 H, I, act, eps, out_dtype)
+        return out
+    return block
+
+
+@pytest.mark.parametrize("kind", ["norms_swapped", "qkv_from_attn_out", "ffn_from_block_input",
+                                  "ffn_norms_swapped"])
+def test_decoder_block_pin_catches_routing_mistakes(kind):
+    with pytest.raises(AssertionError):
+        test_decoder_block_matches_textbook(_block_mutant(kind))
+
+
 def test_decoder_block_runs_and_chains():
     sh = workloads.BlockShape("tiny", hidden=256, n_q=256, n_kv=128, inter=384, act="relu2")
     d = workloads.block_inputs(sh, T=2, seed=3)
@@ -382,7 +483,7 @@ def _sequential_interleave(codes):
     return ((c[:, 0] << 6) | (c[:, 1] << 4) | (c[:, 2] << 2) | c[:, 3]).astype(np.uint8)
 
 
-@pytest.mark.parametrize("mutant", ["sequential_layout", "codes_minus_one", "no_half_even",
+@pytest.mark.parametrize("mutant", ["sequential_layout", "codes_minus_one", "no_half_even", "half_away_from_zero",
                                     "mean_without_divide", "transposed_dot", "gate_up_swapped"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     if mutant == "sequential_layout":
@@ -395,6 +496,9 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     elif mutant == "no_half_even":
         monkeypatch.setattr(O.np, "rint", lambda v: np.floor(np.asarray(v) + 0.5))
         check = test_quant_ties_round_half_even
+    elif mutant == "half_away_from_zero":
+        monkeypatch.setattr(O.np, "rint", lambda v: np.sign(v) * np.floor(np.abs(np.asarray(v)) + 0.5))
+        check = test_ties_of_codes_and_activations_round_half_even
     elif mutant == "mean_without_divide":
         monkeypatch.setattr(O, "fixed_point_mean_f32",
                             lambda t: F32(math.ldexp(float(O.fixed_point_sum(t)[0]), -O.fixed_point_sum(t)[1])))

@@ -11,6 +11,7 @@ import ternary_bitlinear_quantized_b200 as tb
 import workloads
 from oracle import bitnet_oracle as O
 from tests.parity_util import act_to_np, assert_close, bf16_to_np, oracle_rows, out_to_np
+from tests.tie_inputs import tie_activations, tie_weights
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -126,6 +127,53 @@ def test_quant_bitexact(T, K, dtype, use_gain, outliers):
     assert np.array_equal(q.cpu().numpy(), rq)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     assert np.array_equal(sq.cpu().numpy(), rsq)
+
+
+# ----------------------------------------------------------------------------- rounding ties
+
+def test_pack_ties_bitexact():
+    """Weights at exactly +-0.5 and +-1.5 times beta (beta = 2**-6): the codes take the
+    half-to-even decision, so a kernel that rounds half away from zero differs here."""
+    W = tie_weights(N=160, K=256)
+    got = gpu_pack(torch.from_numpy(W)).cpu().numpy()
+    ref = O.pack_i2s(W)
+    assert np.array_equal(got, ref)
+    codes, beta = O.unpack_i2s(got, 160, 256)
+    assert beta == np.float32(2.0 ** -6)
+    assert np.array_equal(codes.astype(np.int16) - 1, np.where(np.abs(W) < 2.0 ** -6, 0, np.sign(W)).astype(np.int16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quant_ties_bitexact(dtype):
+    """Activations (n + 1/2)/64 with absmax 127/64 (s_x = 64): every entry is a .5 tie."""
+    x = tie_activations()
+    xt = torch.from_numpy(x).to(dtype)
+    assert np.array_equal(act_to_np(xt), x)  # exact in bf16
+    q, s, sq = tb.rmsnorm_quant_act(xt.to(DEV), None, 1e-6)
+    rq, rs, rsq = O.rmsnorm_quant_act(x, None, 1e-6)
+    assert np.all(rs == np.float32(64.0))
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(sq.cpu().numpy(), rsq)
+
+
+@pytest.mark.parametrize("reps", [1, 14])  # 3 tokens (decode engine) and 42 (tensor-core path)
+def test_bitlinear_ties_bitexact(reps):
+    """Tie activations through the product with tie weights: q, codes, int32 accumulators and
+    outputs against the oracle, bit for bit."""
+    x = np.tile(tie_activations(), (reps, 1))
+    T, K = x.shape
+    W = tie_weights(N=160, K=K)
+    packed_ref = O.pack_i2s(W)
+    packed = gpu_pack(torch.from_numpy(W))
+    assert np.array_equal(packed.cpu().numpy(), packed_ref)
+    q, s, sq = tb.rmsnorm_quant_act(torch.from_numpy(x).to(torch.bfloat16).to(DEV), None, 1e-6)
+    acc = torch.empty(T, 160, dtype=torch.int32, device=DEV)
+    out = tb.bitlinear(q, s, sq, packed, 160, torch.float32, acc_debug=acc)
+    rq, rs, rsq = O.rmsnorm_quant_act(x, None, 1e-6)
+    ref, racc = O.bitlinear(rq, rs, rsq, packed_ref, 160, K, "f32", return_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
 
 
 # ----------------------------------------------------------------------------- a3/a4: product
