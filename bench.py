@@ -1,9 +1,11 @@
 """Benchmark of the BitNet b1.58 BitLinear forward on B200.
 
-Default workload: the 2B4T-shaped decoder block at decode (T = 1): q,k,v (attn_norm,
-one grouped launch), o (attn_sub_norm, on a synthetic attention output), and the FFN
-(ffn_norm -> gate/up -> relu2 -> ffn_sub_norm -> down, fed by o's output).  A step is
-one pass of that whole path; weights are packed once before timing (offline step).
+Default workload: the 70B-shaped decoder block projections at decode (T = 1): q,k,v
+(attn_norm), o (attn_sub_norm, on a synthetic attention output), and the SiLU FFN
+(ffn_norm -> gate/up -> SiLU -> ffn_sub_norm -> down, fed by o's output), the largest
+configuration that runs on one GPU.  A step is one pass of that whole path; weights are
+packed once before timing (offline step).  The same JSON line carries a `prefill` object
+for the prefill half of the metric: the 32B-shaped FFN block at T = 4096 (int8 TOPS).
 
 value  = packed-weight bytes read per step x steps x ranks / device time (max over ranks)
          [GB/s]; for prefill workloads (T >= 64) int8 TOPS = 2 T sum(N K) / time.
@@ -46,7 +48,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="block_2b4t_decode_t1", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="proj_70b_decode_t1", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--prefill-workload", default="ffn_32b_t4096", choices=sorted(workloads.WORKLOADS) + ["none"],
+                    help="prefill workload reported in the line's `prefill` object ('none' to skip)")
+    ap.add_argument("--prefill-steps", type=int, default=30)
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle sample")
     ap.add_argument("--seed", type=int, default=0)
@@ -340,31 +345,80 @@ def time_steps(wl: Workload, steps: int, warmup: int, use_graph: bool, e2e: bool
     return ms, h2d, d2h
 
 
-def time_dominant(wl: Workload, launches: int):
-    """Average device duration of the dominant kernel, launched alone (weights rotating)."""
+def time_dominant(wl: Workload, steps: int, step_ms: float):
+    """Average device duration (ms) of one launch of the dominant kernel, timed the way the
+    step is timed: CUDA graphs replayed back to back on one stream, weights rotating.  At
+    decode the step IS one launch of the decode engine, so its time is the step's."""
     label, fn, nbytes, ops = wl.dominant()
+    if wl.kind != "bitlinear" and wl.T <= 16:
+        return label, step_ms, nbytes, ops
     R = wl.n_copies
-    for c in range(min(R, 3)):
+    for c in range(min(R, 2)):
         fn(c)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
-    stream = torch.cuda.current_stream()
-    # Hold the GPU while the host enqueues, so that no host launch latency falls between
-    # an event pair; the events also keep consecutive launches from overlapping.
-    torch.cuda._sleep(int(launches * 60_000))
-    for i, (a, b) in enumerate(evs):
-        a.record(stream)
-        fn(i % R)
-        b.record(stream)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for c in range(R):
+            fn(c)
     torch.cuda.synchronize()
-    ms = [a.elapsed_time(b) for a, b in evs]
-    return label, statistics.mean(ms), nbytes, ops
+    reps = max(1, steps // R)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * R)
+    del g
+    return label, ms, nbytes, ops
+
+
+def int8_peak_probe():
+    """Dense int8 tensor-core throughput of this GPU, measured now: torch._int_mm (cuBLASLt,
+    int8 x int8 -> int32) at 8192^3, best of 10 launches after 3 warm-up ones (TOPS)."""
+    n = 8192
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    A = torch.randint(-128, 127, (n, n), dtype=torch.int8, device="cuda", generator=gen)
+    B = torch.randint(-128, 127, (n, n), dtype=torch.int8, device="cuda", generator=gen).t().contiguous().t()
+    for _ in range(3):
+        torch._int_mm(A, B)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(A, B)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        best = ms if best is None else min(best, ms)
+    del A, B
+    return 2.0 * n ** 3 / (best / 1e3) / 1e12
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
-def oracle_sample(name: str, seed: int, seconds: float):
-    """Time the numpy oracle on this workload (bounded sample).  Returns (units/s, unit, sample, cores)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(name: str, seed: int, seconds: float, single_thread_seconds: float = 0.0):
+    """Time the numpy oracle on this workload (bounded sample) on all the host threads numpy
+    uses, and optionally single-threaded.  Returns a dict: value, unit, sample, cores,
+    and (if asked) single_thread_value."""
     import numpy as np
     from oracle import bitnet_oracle as O
     spec = workloads.WORKLOADS[name]
@@ -378,7 +432,8 @@ def oracle_sample(name: str, seed: int, seconds: float):
         xf = O.bf16_bits_to_f32(x.view(torch.int16).numpy().view(np.uint16))
         g = workloads.gain(K, seed, name + "/g").numpy()
         tensors = {"w": (N, K)}
-        run = lambda xs: O.bitlinear_from_x(xs, g, workloads.EPS, packed, N, K, "bf16")
+        run = lambda xs, a=None: O.bitlinear_from_x(xs, g, workloads.EPS, packed, N, K, "bf16")
+        af = None
     else:
         sh = spec["shape"]
         ffn_only = spec["kind"] == "ffn"
@@ -400,35 +455,106 @@ def oracle_sample(name: str, seed: int, seconds: float):
     # Tokens are independent through every step, so a prefill sample takes a few tokens.
     t_sample = T if decode else min(T, 8)
     xs = xf[:t_sample]
-    a_s = None if spec["kind"] != "block" else af[:t_sample]
-    n, t0 = 0, time.perf_counter()
-    while True:
-        if spec["kind"] == "block":
+    a_s = None if af is None else af[:t_sample]
+
+    def timed(limit):
+        n, t0 = 0, time.perf_counter()
+        while True:
             run(xs, a_s)
-        else:
-            run(xs)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= limit:
+                return n, el
+
+    def rate(n, el):
+        if decode:
+            return pbytes * n / el / 1e9
+        return sum(2 * t_sample * nn * kk for (nn, kk) in tensors.values()) * n / el / 1e12
+
+    n, el = timed(seconds)
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = 1
+    out = {"value": rate(n, el), "unit": "GB/s" if decode else "TOPS", "cores": cores, "kind": "oracle",
+           "cpu_model": cpu_model()}
     if decode:
-        val = pbytes * n / el / 1e9
-        unit = "GB/s"
-        sample = f"{n} full steps of the workload (T={T}) in {el:.1f} s"
+        out["sample"] = f"{n} full steps of the workload (T={T}) in {el:.1f} s on {cores} threads"
     else:
-        ops = sum(2 * t_sample * nn * kk for (nn, kk) in tensors.values())
-        val = ops * n / el / 1e12
-        unit = "TOPS"
-        sample = f"{n} steps on {t_sample} of the {T} tokens (tokens are independent) in {el:.1f} s"
-    return val, unit, sample, cores
+        out["sample"] = f"{n} steps on {t_sample} of the {T} tokens (tokens are independent) in {el:.1f} s"
+    if single_thread_seconds > 0:
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                n1, el1 = timed(single_thread_seconds)
+            out["single_thread_value"] = rate(n1, el1)
+            out["single_thread_sample"] = f"{n1} steps in {el1:.1f} s on 1 thread"
+        except Exception as e:  # threadpoolctl missing: report why
+            out["single_thread_value"] = None
+            out["single_thread_sample"] = f"not measured: {e}"
+    return out
 
 
 # ----------------------------------------------------------------------------- main
+
+def roofline(wl: Workload, name: str, label: str, dom_ms: float, dom_bytes: int, dom_ops: int, int8_peak):
+    """The `roofline` object of the dominant kernel (decode: HBM-bound on packed bytes;
+    prefill: int8 tensor-core bound)."""
+    hbm, bf16, src = peaks()
+    decode = wl.T < 64
+    kernel_files = (["ternary_bitlinear_quantized_b200/csrc/engine.cuh"] if decode else
+                    ["ternary_bitlinear_quantized_b200/csrc/gemm_tc.cuh"]) + [
+        "ternary_bitlinear_quantized_b200/csrc/gemv.cuh", "ternary_bitlinear_quantized_b200/csrc/common.cuh"]
+    traffic = stored_traffic(f"{label} @ {name}", source_sha(kernel_files))
+    if decode:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "kernel": label, "bytes_per_launch": dom_bytes, "launch_us": dom_ms * 1e3,
+                "peak_source": f"{src} hbm_gbs (copy bandwidth, burst)"}
+    achieved = dom_ops / (dom_ms / 1e3) / 1e12
+    nominal = bf16 * 2.0  # dense int8 = 2x dense bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
+    peak = int8_peak if int8_peak else nominal
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS", "frac": achieved / peak,
+            "traffic": traffic, "kernel": label, "ops_per_launch": dom_ops, "launch_us": dom_ms * 1e3,
+            "peak_source": ("int8 dense measured in this run (torch._int_mm, cuBLASLt, 8192^3, best of 10)"
+                            if int8_peak else f"{src} bf16_tflops x 2 (nominal int8/bf16 ratio)"),
+            "frac_of_bf16x2": achieved / nominal}
+
+
+def measure(name: str, args, world: int, use_graph: bool, steps: int, int8_peak=None):
+    """Device-timed throughput, end-to-end throughput and the dominant kernel of one
+    workload (max over ranks).  Returns (line fields, clocks)."""
+    spec = workloads.WORKLOADS[name]
+    decode = spec["T"] < 64
+    wl = Workload(name, args.seed + 0, f"cuda:{torch.cuda.current_device()}")  # same workload on every rank
+    clk = ClockSampler(torch.cuda.current_device())
+    clk.start()
+    ms, _, _ = time_steps(wl, steps, args.warmup, use_graph, e2e=False)
+    clocks = clk.stop()
+    ms_e2e, h2d, d2h = time_steps(wl, steps, args.warmup, use_graph, e2e=True)
+    label, dom_ms, dom_bytes, dom_ops = time_dominant(wl, steps, ms / steps)
+    status = wl.tb.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    ms, ms_e2e, dom_ms = max_over_ranks([ms, ms_e2e, dom_ms])
+    per_step_units = wl.packed_bytes / 1e9 if decode else wl.ops_per_step / 1e12
+    fields = {
+        "metric": "packed-weight HBM GB/s (decode)" if decode else "int8 TOPS (prefill)",
+        "value": whole_job_rate(per_step_units, steps, world, ms),
+        "unit": "GB/s" if decode else "TOPS",
+        "steps": steps,
+        "ms_per_step": ms / steps,
+        "config": workload_config(name, world, use_graph),
+        "roofline": roofline(wl, name, label, dom_ms, dom_bytes, dom_ops, int8_peak),
+        "e2e": {"value": whole_job_rate(per_step_units, steps, world, ms_e2e), "unit": "GB/s" if decode else "TOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": wl.launches_per_step() * steps,
+    }
+    del wl
+    torch.cuda.empty_cache()
+    return fields, clocks
+
 
 def main():
     args = parse()
@@ -438,17 +564,17 @@ def main():
     spec = workloads.WORKLOADS[args.workload]
     decode = spec["T"] < 64
     metric = ("packed-weight HBM GB/s (decode)" if decode else "int8 TOPS (prefill)")
-    unit = "GB/s" if decode else "TOPS"
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        val, u, sample, cores = oracle_sample(args.workload, args.seed, args.cpu_seconds)
+        cpu = oracle_sample(args.workload, args.seed, args.cpu_seconds)
+        val, u = cpu["value"], cpu["unit"]
         line = {"metric": metric, "value": val, "unit": u, "n_gpus": args.gpus, "steps": args.steps,
                 "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "impl": "reference", "dtype": "int8", "data": "synthetic",
                 "config": workload_config(args.workload, args.gpus, not args.no_graph),
-                "cpu_baseline": {"value": val, "unit": u, "cores": cores, "kind": "oracle", "sample": sample},
+                "cpu_baseline": cpu,
                 "e2e": {"value": val, "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
@@ -463,59 +589,39 @@ def main():
         tbuild.build()
     if world > 1:
         torch.distributed.barrier()
-    wl = Workload(args.workload, args.seed + 0, f"cuda:{local}")  # same workload on every rank (replicas)
     use_graph = not args.no_graph
 
-    clk = ClockSampler(local)
-    clk.start()
-    ms, _, _ = time_steps(wl, args.steps, args.warmup, use_graph, e2e=False)
-    clocks = clk.stop()
-    ms_e2e, h2d, d2h = time_steps(wl, args.steps, args.warmup, use_graph, e2e=True)
-    label, dom_ms, dom_bytes, dom_ops = time_dominant(wl, max(50, min(args.steps, 500)))
-    status = wl.tb.device_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status}")
-
-    ms, ms_e2e = max_over_ranks([ms, ms_e2e])
-    per_step_units = wl.packed_bytes / 1e9 if decode else wl.ops_per_step / 1e12
-    value = whole_job_rate(per_step_units, args.steps, world, ms)
-    e2e_val = whole_job_rate(per_step_units, args.steps, world, ms_e2e)
-
-    hbm, bf16, src = peaks()
-    kernel_files = (["ternary_bitlinear_quantized_b200/csrc/engine.cuh"] if decode else
-                    ["ternary_bitlinear_quantized_b200/csrc/gemm_tc.cuh"]) + [
-        "ternary_bitlinear_quantized_b200/csrc/gemv.cuh", "ternary_bitlinear_quantized_b200/csrc/common.cuh"]
-    if decode:
-        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": stored_traffic(f"{label} @ {args.workload}", source_sha(kernel_files)), "kernel": label,
-                "bytes_per_launch": dom_bytes, "launch_us": dom_ms * 1e3,
-                "peak_source": f"{src} hbm_gbs (copy bandwidth, burst)"}
-    else:
-        achieved = dom_ops / (dom_ms / 1e3) / 1e12
-        int8_peak = bf16 * 2.0  # dense int8 = 2x dense bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
-        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak,
-                "traffic": stored_traffic(f"{label} @ {args.workload}", source_sha(kernel_files)), "kernel": label,
-                "ops_per_launch": dom_ops, "launch_us": dom_ms * 1e3,
-                "peak_source": f"{src} bf16_tflops x 2 (nominal int8/bf16 ratio)"}
+    main_fields, clocks = measure(args.workload, args, world, use_graph, args.steps)
+    prefill = None
+    if args.prefill_workload != "none":
+        pspec = workloads.WORKLOADS[args.prefill_workload]
+        int8_peak = int8_peak_probe() if pspec["T"] >= 64 else None
+        pf, pclocks = measure(args.prefill_workload, args, world, use_graph, args.prefill_steps, int8_peak)
+        prefill = {"workload": args.prefill_workload, **{k: pf[k] for k in
+                   ("metric", "value", "unit", "steps", "ms_per_step", "config", "roofline", "e2e", "gpu_launches")},
+                   "clocks": pclocks, "int8_peak_measured_tops": int8_peak}
 
     cpu = None
     if rank == 0 and world == 1:
-        val, u, sample, cores = oracle_sample(args.workload, args.seed, args.cpu_seconds)
-        cpu = {"value": val, "unit": u, "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = oracle_sample(args.workload, args.seed, args.cpu_seconds, single_thread_seconds=args.cpu_seconds / 2)
+        if prefill is not None:
+            prefill["cpu_baseline"] = oracle_sample(args.prefill_workload, args.seed, args.cpu_seconds / 2,
+                                                    single_thread_seconds=args.cpu_seconds / 4)
 
     if rank == 0:
         line = {
-            "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": workload_config(args.workload, world, use_graph),
-            "roofline": roof,
+            "metric": main_fields["metric"], "value": main_fields["value"], "unit": main_fields["unit"],
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_fields["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": main_fields["config"],
+            "roofline": main_fields["roofline"],
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": wl.launches_per_step() * args.steps,
+            "e2e": main_fields["e2e"],
+            "gpu_launches": main_fields["gpu_launches"],
             "clocks": clocks,
         }
+        if prefill is not None:
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

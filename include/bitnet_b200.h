@@ -150,6 +150,47 @@ bitnet_status bitnet_bitlinear_gate_up_act(const int8_t* q, const float* s_x, co
                                            int64_t I, int64_t K, bitnet_act act, float* h,
                                            bitnet_stream s);
 
+/* The integer part of bitnet_bitlinear only: acc[t, n] = sum_k q[t, k] * c[n, k] - sum_q[t]
+ * (int32 [T, N]); no scale is read and no float output is written.  With the activation
+ * sum of a slice of the in-features (sum_q of that slice) and an I2_S tensor holding only
+ * those in-features, acc is that slice's share of the product, and the shares of disjoint
+ * slices add up exactly to the full product (tensor parallelism over K).  [I2S] "I2_S NEON
+ * kernel for the canonical layout".  Errors: NULL, SHAPE, ALIGN. */
+bitnet_status bitnet_bitlinear_acc(const int8_t* q, const int32_t* sum_q, const uint8_t* packed, int64_t T,
+                                   int64_t N, int64_t K, int32_t* acc, bitnet_stream s);
+
+/* out[t, n] = fp32(acc[t, n]) * (beta / s_x[t]) with beta from the trailer of `packed` (an I2_S
+ * tensor of N x K weights): the dequantising epilogue of bitnet_bitlinear applied to int32
+ * accumulators that were summed over ranks.  out: bf16 (nearest even) or fp32 [T, N].
+ * Errors: NULL, SHAPE, ALIGN (packed), DTYPE. */
+bitnet_status bitnet_dequant_acc(const int32_t* acc, const float* s_x, const uint8_t* packed, int64_t T,
+                                 int64_t N, int64_t K, void* out, bitnet_dtype ot, bitnet_stream s);
+
+/* ffn_sub_norm + absmax int8 of h [T, K_total] when each rank holds Ks of its columns (h [T, Ks]
+ * fp32 here, the rank's gate/up shard; gain: the matching Ks entries of ffn_sub_norm or NULL).
+ * Every reduction of the norm is exact (maxima and an integer fixed-point sum), so it is
+ * finished over the ranks by all-reduces, and the result is bit-identical to the unsharded
+ * bitnet_rmsnorm_quant_act of the whole row:
+ *   shard_amax    amax[t] = max |h[t, :]| over this shard          -> all-reduce MAX over ranks
+ *   shard_sumsq   S[t] = sum rint(h^2 2^e) over this shard, on the grid e of the whole row
+ *                 (from the GLOBAL amax and K_total)                -> all-reduce SUM (int64)
+ *   shard_ymax    inv[t] = 1/sqrt(mean + eps) (mean = fp32(S 2^-e / K_total)), and
+ *                 ymax[t] = max |(h inv) gain| over this shard      -> all-reduce MAX
+ *                 (gain NULL: inv = 1, ymax = the global amax; S is not read)
+ *   shard_quant   s_x[t] = 127 / max(ymax, 1e-5) (global ymax), q = clamp(rint(y s_x)) [T, Ks],
+ *                 sum_q[t] = this shard's sum of q (the shard's activation sum)
+ * [RMS] BitNetMLP.forward (ffn_sub_norm over the whole intermediate row).  Per-token
+ * arrays (amax, inv, ymax, s_x: fp32 [T]; S: int64 [T], 8-byte aligned; sum_q: int32 [T]) are
+ * device memory.  Ks % 4 == 0; h, gain, q 16-byte aligned.  Errors: NULL, SHAPE, ALIGN. */
+bitnet_status bitnet_subnorm_shard_amax(const float* h, int64_t T, int64_t Ks, float* amax, bitnet_stream s);
+bitnet_status bitnet_subnorm_shard_sumsq(const float* h, int64_t T, int64_t Ks, const float* amax, int64_t K_total,
+                                         int64_t* S, bitnet_stream s);
+bitnet_status bitnet_subnorm_shard_ymax(const float* h, const float* gain, int64_t T, int64_t Ks, const float* amax,
+                                        const int64_t* S, int64_t K_total, float eps, float* inv, float* ymax,
+                                        bitnet_stream s);
+bitnet_status bitnet_subnorm_shard_quant(const float* h, const float* gain, int64_t T, int64_t Ks, const float* inv,
+                                         const float* ymax, int8_t* q, float* s_x, int32_t* sum_q, bitnet_stream s);
+
 /* Workspace of bitnet_ffn_block, in bytes (0 if a size is invalid). */
 size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I);
 

@@ -61,14 +61,27 @@ ABS_FLOOR = F32(1e-5)  # the 1e-5 floor of both absmax and absmean
 
 # ----------------------------------------------------------------------------- sums
 
-def fixed_point_sum(terms: np.ndarray) -> tuple[int, int]:
-    """Order-free sum of non-negative fp64 ``terms`` on a fixed-point grid.
+def fixed_point_grid(M: float, n: int) -> int:
+    """Grid exponent e of an order-free sum of n non-negative terms whose largest is M > 0:
+    with M = m 2**E (0.5 <= m < 1) and 2**L >= n, e = 62 - E - L, so that every scaled term
+    is below 2**(62 - L) and n of them sum below 2**62 in int64."""
+    _, E = math.frexp(float(M))
+    L = (int(n) - 1).bit_length()
+    return 62 - E - L
 
-    With M = max(terms) = m 2**E (0.5 <= m < 1) and 2**L >= n, the grid step is
-    2**-e with e = 62 - E - L: every term is below 2**(62 - L), so n of them sum below
-    2**62 in int64.  Each term is scaled by 2**e (exact) and rounded half-to-even to an
-    integer; the integer sum S is the same in any order.  Returns (S, e).
-    """
+
+def fixed_point_sum_on_grid(terms: np.ndarray, e: int) -> int:
+    """Sum of rint(term * 2**e) over ``terms`` (each scaled exactly, rounded half-to-even to
+    an integer); the integer sum is the same in any order and over any split of the terms."""
+    terms = np.asarray(terms, dtype=F64).ravel()
+    if terms.size == 0:
+        return 0
+    return int(np.rint(np.ldexp(terms, e)).astype(np.int64).sum(dtype=np.int64))
+
+
+def fixed_point_sum(terms: np.ndarray) -> tuple[int, int]:
+    """Order-free sum of non-negative fp64 ``terms`` on the fixed-point grid of
+    ``fixed_point_grid(max(terms), n)``.  Returns (S, e)."""
     terms = np.asarray(terms, dtype=F64).ravel()
     n = terms.size
     if n == 0:
@@ -76,11 +89,8 @@ def fixed_point_sum(terms: np.ndarray) -> tuple[int, int]:
     M = float(terms.max())
     if M == 0.0:
         return 0, 0
-    _, E = math.frexp(M)
-    L = (n - 1).bit_length()
-    e = 62 - E - L
-    ints = np.rint(np.ldexp(terms, e)).astype(np.int64)
-    return int(ints.sum(dtype=np.int64)), e
+    e = fixed_point_grid(M, n)
+    return fixed_point_sum_on_grid(terms, e), e
 
 
 def fixed_point_mean_f32(terms: np.ndarray) -> np.float32:
@@ -230,6 +240,68 @@ def rmsnorm_quant_act(x: np.ndarray, gain: np.ndarray | None, eps: float):
         s_x[t] = s
     sum_q = q.astype(np.int64).sum(axis=1).astype(np.int32)
     return q, s_x, sum_q
+
+
+# ----------------------------------------------------------------------------- a6 split over ranks
+
+# ffn_sub_norm when each rank holds some columns of h (tensor parallelism over the FFN's
+# intermediate dimension, the split the gate/up projections produce).  The same arithmetic
+# as rmsnorm_quant_act, taken in stages whose partial results are combined over the ranks
+# by maxima and integer sums; the combination is exact, so the result equals
+# rmsnorm_quant_act of the whole row.
+
+def shard_amax(h: np.ndarray) -> np.ndarray:
+    """max |h| of each row of this shard (combined over ranks by a maximum)."""
+    h = np.atleast_2d(np.asarray(h, dtype=F32))
+    return np.max(np.abs(h), axis=1) if h.shape[1] else np.zeros(h.shape[0], F32)
+
+
+def shard_sumsq(h: np.ndarray, amax: np.ndarray, n_total: int) -> np.ndarray:
+    """This shard's part of the fixed-point sum of h^2 on the grid of the whole row (from
+    the global max |h| and the global row length); combined over ranks by a sum."""
+    h = np.atleast_2d(np.asarray(h, dtype=F32))
+    out = np.zeros(h.shape[0], dtype=np.int64)
+    for t in range(h.shape[0]):
+        a = float(amax[t])
+        if a > 0.0:
+            e = fixed_point_grid(a * a, n_total)
+            out[t] = fixed_point_sum_on_grid(h[t].astype(F64) * h[t].astype(F64), e)
+    return out
+
+
+def shard_ymax(h, gain, amax, S, n_total: int, eps: float):
+    """inv = 1 / sqrt(mean(h^2) + eps) of the whole row (from the combined sum) and this
+    shard's max |y|, y = (h * inv) * g (no gain: inv = 1 and y = h).  Returns (inv, ymax)."""
+    h = np.atleast_2d(np.asarray(h, dtype=F32))
+    T = h.shape[0]
+    inv = np.ones(T, dtype=F32)
+    ymax = np.zeros(T, dtype=F32)
+    for t in range(T):
+        if gain is None:
+            ymax[t] = amax[t]
+            continue
+        a = float(amax[t])
+        ms = F32(0.0)
+        if a > 0.0 and S[t] != 0:
+            e = fixed_point_grid(a * a, n_total)
+            ms = F32(math.ldexp(float(S[t]), -e) / float(n_total))
+        inv[t] = F32(1.0) / np.sqrt(ms + F32(eps))
+        y = (h[t] * inv[t]) * np.asarray(gain, dtype=F32)
+        ymax[t] = np.max(np.abs(y)) if y.size else F32(0.0)
+    return inv, ymax
+
+
+def shard_quant(h, gain, inv, ymax):
+    """s_x = 127 / max(global max |y|, 1e-5); this shard's q and its partial sum of q."""
+    h = np.atleast_2d(np.asarray(h, dtype=F32))
+    T, Ks = h.shape
+    q = np.zeros((T, Ks), dtype=np.int8)
+    s = np.zeros(T, dtype=F32)
+    for t in range(T):
+        y = h[t] if gain is None else (h[t] * F32(inv[t])) * np.asarray(gain, dtype=F32)
+        s[t] = F32(127.0) / np.maximum(F32(ymax[t]), ABS_FLOOR)
+        q[t] = np.clip(np.rint(y * s[t]), -128, 127).astype(np.int8)
+    return q, s, q.astype(np.int64).sum(axis=1).astype(np.int32)
 
 
 # ----------------------------------------------------------------------------- a3/a4: dot + dequant

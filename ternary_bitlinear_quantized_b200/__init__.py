@@ -68,6 +68,12 @@ def lib() -> ctypes.CDLL:
         "bitnet_bitlinear": (c_i, [c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i, c_p, c_p]),
         "bitnet_bitlinear_group": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_i64, c_i64, c_p, c_i, c_p]),
         "bitnet_bitlinear_gate_up_act": (c_i, [c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_p, c_p]),
+        "bitnet_bitlinear_acc": (c_i, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_p]),
+        "bitnet_dequant_acc": (c_i, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_i, c_p]),
+        "bitnet_subnorm_shard_amax": (c_i, [c_p, c_i64, c_i64, c_p, c_p]),
+        "bitnet_subnorm_shard_sumsq": (c_i, [c_p, c_i64, c_i64, c_p, c_i64, c_p, c_p]),
+        "bitnet_subnorm_shard_ymax": (c_i, [c_p, c_p, c_i64, c_i64, c_p, c_p, c_i64, c_f, c_p, c_p, c_p]),
+        "bitnet_subnorm_shard_quant": (c_i, [c_p, c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_p, c_p]),
         "bitnet_ffn_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64]),
         "bitnet_ffn_workspace_offsets": (c_i, [c_i64, c_i64, c_i64, c_p]),
         "bitnet_ffn_block": (c_i, [c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_i,
@@ -187,6 +193,66 @@ def bitlinear(q, s_x, sum_q, packed, N: int, out_dtype=torch.bfloat16, out=None,
     _check(lib().bitnet_bitlinear(_ptr(q), _ptr(s_x), _ptr(sum_q), _ptr(packed), T, N, K, _ptr(out),
                                   _dtype_code(out.dtype), _ptr(acc_debug), _stream(stream)), "bitlinear")
     return out
+
+
+def bitlinear_acc(q, sum_q, packed, N: int, out=None, stream=None) -> torch.Tensor:
+    """int32 accumulators [T, N] = q @ c^T - sum_q (no dequantisation)."""
+    T, K = q.shape
+    for t, nm in ((q, "q"), (sum_q, "sum_q"), (packed, "packed")):
+        _need(t, nm)
+    acc = out if out is not None else torch.empty(T, N, dtype=torch.int32, device=q.device)
+    _check(lib().bitnet_bitlinear_acc(_ptr(q), _ptr(sum_q), _ptr(packed), T, N, K, _ptr(acc), _stream(stream)),
+           "bitlinear_acc")
+    return acc
+
+
+def dequant_acc(acc, s_x, packed, K: int, out_dtype=torch.bfloat16, out=None, stream=None) -> torch.Tensor:
+    """out = fp32(acc) * (beta / s_x), beta from the I2_S trailer of `packed` ([N, K])."""
+    T, N = acc.shape
+    for t, nm in ((acc, "acc"), (s_x, "s_x"), (packed, "packed")):
+        _need(t, nm)
+    o = out if out is not None else torch.empty(T, N, dtype=out_dtype, device=acc.device)
+    _check(lib().bitnet_dequant_acc(_ptr(acc), _ptr(s_x), _ptr(packed), T, N, K, _ptr(o), _dtype_code(o.dtype),
+                                    _stream(stream)), "dequant_acc")
+    return o
+
+
+def subnorm_shard_amax(h, out=None, stream=None):
+    T, Ks = h.shape
+    _need(h, "h")
+    a = out if out is not None else torch.empty(T, dtype=torch.float32, device=h.device)
+    _check(lib().bitnet_subnorm_shard_amax(_ptr(h), T, Ks, _ptr(a), _stream(stream)), "subnorm_shard_amax")
+    return a
+
+
+def subnorm_shard_sumsq(h, amax, K_total: int, out=None, stream=None):
+    T, Ks = h.shape
+    _need(h, "h")
+    S = out if out is not None else torch.empty(T, dtype=torch.int64, device=h.device)
+    _check(lib().bitnet_subnorm_shard_sumsq(_ptr(h), T, Ks, _ptr(amax), K_total, _ptr(S), _stream(stream)),
+           "subnorm_shard_sumsq")
+    return S
+
+
+def subnorm_shard_ymax(h, gain, amax, S, K_total: int, eps: float = 1e-6, stream=None):
+    T, Ks = h.shape
+    _need(h, "h")
+    inv = torch.empty(T, dtype=torch.float32, device=h.device)
+    ymax = torch.empty(T, dtype=torch.float32, device=h.device)
+    _check(lib().bitnet_subnorm_shard_ymax(_ptr(h), _ptr(gain), T, Ks, _ptr(amax), _ptr(S), K_total, eps, _ptr(inv),
+                                           _ptr(ymax), _stream(stream)), "subnorm_shard_ymax")
+    return inv, ymax
+
+
+def subnorm_shard_quant(h, gain, inv, ymax, stream=None):
+    T, Ks = h.shape
+    _need(h, "h")
+    q = torch.empty(T, Ks, dtype=torch.int8, device=h.device)
+    s = torch.empty(T, dtype=torch.float32, device=h.device)
+    sq = torch.empty(T, dtype=torch.int32, device=h.device)
+    _check(lib().bitnet_subnorm_shard_quant(_ptr(h), _ptr(gain), T, Ks, _ptr(inv), _ptr(ymax), _ptr(q), _ptr(s),
+                                            _ptr(sq), _stream(stream)), "subnorm_shard_quant")
+    return q, s, sq
 
 
 def bitlinear_group(q, s_x, sum_q, packed: list, Ns: list, out_dtype=torch.bfloat16, outs=None, stream=None):

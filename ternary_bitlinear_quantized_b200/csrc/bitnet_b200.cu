@@ -14,6 +14,7 @@
 #include "gemv.cuh"
 #include "engine.cuh"
 #include "gemm_tc.cuh"
+#include "shard.cuh"
 
 namespace bitnet {
 
@@ -603,6 +604,100 @@ bitnet_status bitnet_bitlinear_gate_up_act(const int8_t* q, const float* s_x, co
   const int64_t nI[2] = {I, I};
   return enqueue_gemv(q, s_x, sum_q, 2, gu, nI, nullptr, nullptr, T, K, BITNET_F32, true, act, h,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_bitlinear_acc(const int8_t* q, const int32_t* sum_q, const uint8_t* packed, int64_t T, int64_t N,
+                                   int64_t K, int32_t* acc, bitnet_stream stream) {
+  if (T < 0 || K <= 0 || K % 128 != 0 || K > BITNET_MAX_K || T > 0x7FFFFFFFll || N <= 0 || N > (1 << 30))
+    return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!q || !sum_q || !packed || !acc) return BITNET_ERR_NULL;
+  if (!aligned16(q) || !aligned16(sum_q) || !aligned16(packed) || !aligned16(acc)) return BITNET_ERR_ALIGN;
+  const uint8_t* p[1] = {packed};
+  const int64_t n[1] = {N};
+  void* o[1] = {nullptr};
+  int32_t* d[1] = {acc};
+  return enqueue_gemv(q, nullptr, sum_q, 1, p, n, o, d, T, K, BITNET_F32, false, BITNET_RELU2, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- tensor-parallel pieces
+static unsigned shard_grid(int64_t T) {
+  const int64_t cap = (int64_t)device_sm_count() * 8;
+  return (unsigned)(T < cap ? T : cap);
+}
+
+static bitnet_status shard_checks(const float* h, int64_t T, int64_t Ks) {
+  if (T < 0 || T > 0x7FFFFFFFll || Ks <= 0 || Ks % 4 != 0 || Ks > (1 << 30)) return BITNET_ERR_SHAPE;
+  if (T > 0 && !h) return BITNET_ERR_NULL;
+  if (T > 0 && !aligned16(h)) return BITNET_ERR_ALIGN;
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_subnorm_shard_amax(const float* h, int64_t T, int64_t Ks, float* amax, bitnet_stream stream) {
+  bitnet_status st = shard_checks(h, T, Ks);
+  if (st != BITNET_OK || T == 0) return st;
+  if (!amax) return BITNET_ERR_NULL;
+  cudaError_t e = launch(k_shard_amax, dim3(shard_grid(T)), dim3(SHARD_THREADS), 0,
+                         reinterpret_cast<cudaStream_t>(stream), true, h, (int)T, (int)Ks, amax);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_shard_amax");
+}
+
+bitnet_status bitnet_subnorm_shard_sumsq(const float* h, int64_t T, int64_t Ks, const float* amax, int64_t K_total,
+                                         int64_t* S, bitnet_stream stream) {
+  bitnet_status st = shard_checks(h, T, Ks);
+  if (st != BITNET_OK || T == 0) return st;
+  if (K_total < Ks || K_total > (1ll << 40)) return BITNET_ERR_SHAPE;
+  if (!amax || !S) return BITNET_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(S) & 7) return BITNET_ERR_ALIGN;
+  cudaError_t e = launch(k_shard_sumsq, dim3(shard_grid(T)), dim3(SHARD_THREADS), 0,
+                         reinterpret_cast<cudaStream_t>(stream), true, h, (int)T, (int)Ks, amax, (long long)K_total,
+                         reinterpret_cast<long long*>(S));
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_shard_sumsq");
+}
+
+bitnet_status bitnet_subnorm_shard_ymax(const float* h, const float* gain, int64_t T, int64_t Ks, const float* amax,
+                                        const int64_t* S, int64_t K_total, float eps, float* inv, float* ymax,
+                                        bitnet_stream stream) {
+  bitnet_status st = shard_checks(h, T, Ks);
+  if (st != BITNET_OK || T == 0) return st;
+  if (K_total < Ks || K_total > (1ll << 40)) return BITNET_ERR_SHAPE;
+  if (!amax || !inv || !ymax || (gain && !S)) return BITNET_ERR_NULL;
+  if ((gain && !aligned16(gain)) || (reinterpret_cast<uintptr_t>(S) & 7)) return BITNET_ERR_ALIGN;
+  cudaError_t e = launch(k_shard_ymax, dim3(shard_grid(T)), dim3(SHARD_THREADS), 0,
+                         reinterpret_cast<cudaStream_t>(stream), true, h, gain, (int)T, (int)Ks, amax,
+                         reinterpret_cast<const long long*>(S), (long long)K_total, eps, inv, ymax);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_shard_ymax");
+}
+
+bitnet_status bitnet_subnorm_shard_quant(const float* h, const float* gain, int64_t T, int64_t Ks, const float* inv,
+                                         const float* ymax, int8_t* q, float* s_x, int32_t* sum_q,
+                                         bitnet_stream stream) {
+  bitnet_status st = shard_checks(h, T, Ks);
+  if (st != BITNET_OK || T == 0) return st;
+  if (!inv || !ymax || !q || !s_x || !sum_q) return BITNET_ERR_NULL;
+  if ((gain && !aligned16(gain)) || !aligned16(q)) return BITNET_ERR_ALIGN;
+  cudaError_t e = launch(k_shard_quant, dim3(shard_grid(T)), dim3(SHARD_THREADS), 0,
+                         reinterpret_cast<cudaStream_t>(stream), true, h, gain, (int)T, (int)Ks, inv, ymax, q, s_x,
+                         sum_q);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_shard_quant");
+}
+
+bitnet_status bitnet_dequant_acc(const int32_t* acc, const float* s_x, const uint8_t* packed, int64_t T, int64_t N,
+                                 int64_t K, void* out, bitnet_dtype ot, bitnet_stream stream) {
+  if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (T < 0 || T > 0x7FFFFFFFll || N <= 0 || N > (1 << 30) || K <= 0 || K % 128 != 0) return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!acc || !s_x || !packed || !out) return BITNET_ERR_NULL;
+  if (!aligned16(packed)) return BITNET_ERR_ALIGN;
+  const float* beta = reinterpret_cast<const float*>(packed + N * K / 4);
+  const long long total = T * N;
+  const long long want = (total + SHARD_THREADS - 1) / SHARD_THREADS;
+  const long long cap = (long long)device_sm_count() * 8;
+  cudaError_t e = launch(k_dequant_acc, dim3((unsigned)(want < cap ? want : cap)), dim3(SHARD_THREADS), 0,
+                         reinterpret_cast<cudaStream_t>(stream), true, acc, s_x, beta, (long long)T, (int)N, out,
+                         (int)ot);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_dequant_acc");
 }
 
 static size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }

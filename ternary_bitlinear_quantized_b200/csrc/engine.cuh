@@ -901,7 +901,8 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         const long long n = n0 + row;
         const int N = p.t[ti].N;
         const int sq = local ? s_loc_sq[t] : __ldcg(p.sq + t);
-        const float sx = local ? s_loc_s[t] : __ldcg(p.s + t);
+        // s_x may be absent when only the int32 accumulators are asked for (no float output).
+        const float sx = local ? s_loc_s[t] : (p.s != nullptr ? __ldcg(p.s + t) : 1.0f);
         const int* at = acc + tl2 * NT * GEMV_ROWS * T;
         const int accA = at[row * T + t] - sq;
         const float betaA = s_beta[pi][ti];
@@ -914,7 +915,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
           p.h[(long long)t * N + n] = hv;
           if (p.pmax != nullptr) atomicMax(&s_hmax[t], __float_as_uint(fabsf(hv)));
         } else {
-          store_out(p.t[ti].out, p.out_dtype, (long long)t * N + n, vA);
+          if (p.t[ti].out) store_out(p.t[ti].out, p.out_dtype, (long long)t * N + n, vA);
           if (p.t[ti].acc_debug) p.t[ti].acc_debug[(long long)t * N + n] = accA;
         }
       }

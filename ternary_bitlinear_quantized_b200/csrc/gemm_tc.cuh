@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
       // Per-token factors of this tile: beta / s_x and the activation sum.
       for (int j = et; j < BN; j += 128) {
         const int t = tok0 + j;
-        const float sx = t < a.T ? __ldg(a.s_x + t) : 1.0f;
+        const float sx = (t < a.T && a.s_x != nullptr) ? __ldg(a.s_x + t) : 1.0f;  // absent: accumulators only
 #pragma unroll
         for (int u = 0; u < NT; ++u) {
           const uint8_t* pk = a.t[FFN ? u : ti].packed;
@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
             const float vU = dequant(accU, s_f[1][c0 + j]);
             a.h[(long long)t * N + n] = ffn_act(vA, vU, a.act);
           } else {
-            store_out(a.t[ti].out, a.out_dtype, (long long)t * N + n, vA);
+            if (a.t[ti].out) store_out(a.t[ti].out, a.out_dtype, (long long)t * N + n, vA);
             if (a.t[ti].acc_debug) a.t[ti].acc_debug[(long long)t * N + n] = accA;
           }
         }
