@@ -416,3 +416,51 @@ def decoder_block(x, attn_out, gains: dict, packed: dict, shape: dict, act, eps,
     out["ffn"] = ffn_block(out["o"], gains["ffn_norm"], packed["gate"], packed["up"],
                            gains["ffn_sub_norm"], packed["down"], H, I, act, eps, out_dtype)
     return out
+
+
+# ----------------------------------------------------------------------------- the rest of the block
+
+# The attention between the q/k/v and o projections of a decoder block.  The pages keep the
+# transformer's attention and only swap its linear layers for BitLinear ("Add BitNet" in
+# flash-linear-attention: the transformer code with nn.Linear replaced; "More BitNet-like
+# IQ1_S quantizations": per-block attn_q/k/v/output and attn_norm/attn_sub_norm tensors).
+# They do not print it, so it is written here in its textbook form, in fp64: rotary position
+# embedding on q and k (the rotate-half pairing of dimensions i and i + d/2, frequency
+# theta^(-2i/d)), then causal scaled dot-product attention with grouped key/value heads.
+
+def rope_inv_freq(d: int, theta: float) -> np.ndarray:
+    """theta^(-2i/d) for i < d/2, in fp64."""
+    return np.power(float(theta), -2.0 * np.arange(d // 2, dtype=F64) / float(d))
+
+
+def apply_rope(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """x [T, H, d] at token positions [T] -> rotated copy (fp64): for i < d/2,
+    (x_i, x_{i+d/2}) -> (x_i cos a - x_{i+d/2} sin a, x_{i+d/2} cos a + x_i sin a), a = p theta^(-2i/d)."""
+    x = np.asarray(x, dtype=F64)
+    T, H, d = x.shape
+    ang = np.asarray(positions, dtype=F64)[:, None] * rope_inv_freq(d, theta)[None, :]  # [T, d/2]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    x1, x2 = x[..., : d // 2], x[..., d // 2:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray) -> np.ndarray:
+    """Causal grouped-query attention in fp64.  q [T, Hq, d] (already rotated) at positions
+    q_pos [T]; k, v [L, Hkv, d] (keys already rotated) at positions 0..L-1.  Query head h uses
+    key/value head h // (Hq / Hkv); a query at position p sees keys 0..p.  Returns [T, Hq, d]:
+    softmax(q . k / sqrt(d)) v."""
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    v = np.asarray(v, dtype=F64)
+    T, Hq, d = q.shape
+    L, Hkv, _ = k.shape
+    group = Hq // Hkv
+    out = np.zeros((T, Hq, d), dtype=F64)
+    for t in range(T):
+        n = int(q_pos[t]) + 1
+        for h in range(Hq):
+            kh = h // group
+            s = (k[:n, kh, :] @ q[t, h, :]) / math.sqrt(d)
+            w = np.exp(s - s.max())
+            out[t, h] = (w / w.sum()) @ v[:n, kh, :]
+    return out

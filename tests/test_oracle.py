@@ -571,3 +571,97 @@ def test_validate_i2s_counts_planted_faults():
         sc = p.copy()
         sc[nb:nb + 4] = np.frombuffer(np.asarray([val], dtype="<f4").tobytes(), dtype=np.uint8)
         assert O.validate_i2s(sc, 4, 256) == (0, 0, 1), val
+
+
+# ----------------------------------------------------------------------------- rotary embedding, attention
+
+def test_rope_is_identity_at_position_zero_and_preserves_pair_norms():
+    x = np.random.default_rng(1).standard_normal((3, 4, 128))
+    assert np.array_equal(O.apply_rope(x, np.zeros(3), 10000.0), x)
+    y = O.apply_rope(x, np.array([1, 17, 4095]), 10000.0)
+    n_x = x[..., :64] ** 2 + x[..., 64:] ** 2
+    n_y = y[..., :64] ** 2 + y[..., 64:] ** 2
+    assert np.allclose(n_x, n_y, rtol=1e-13, atol=0)
+
+
+def test_rope_equals_complex_rotation():
+    """(x_i + j x_{i+d/2}) e^{j p theta^(-2i/d)}: the rotation written with complex numbers."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 2, 64))
+    pos = np.array([0, 3, 100, 1000, 65535])
+    for theta in (10000.0, 500000.0):
+        z = x[..., :32] + 1j * x[..., 32:]
+        i = np.arange(32)
+        rot = np.exp(1j * pos[:, None, None] * np.power(theta, -2.0 * i / 64.0)[None, None, :])
+        want = np.concatenate([(z * rot).real, (z * rot).imag], axis=-1)
+        assert np.allclose(O.apply_rope(x, pos, theta), want, rtol=0, atol=1e-12)
+
+
+def test_rope_dot_products_depend_on_relative_position_only():
+    rng = np.random.default_rng(3)
+    q, k = rng.standard_normal((1, 1, 128)), rng.standard_normal((1, 1, 128))
+    d0 = float(np.sum(O.apply_rope(q, np.array([7]), 1e4) * O.apply_rope(k, np.array([3]), 1e4)))
+    for shift in (1, 50, 1000):
+        d1 = float(np.sum(O.apply_rope(q, np.array([7 + shift]), 1e4) * O.apply_rope(k, np.array([3 + shift]), 1e4)))
+        assert abs(d1 - d0) <= 1e-9 * (1 + abs(d0))
+
+
+def _sdpa_reference(q, k, v, q_pos):
+    """torch's scaled_dot_product_attention in fp64, with the key/value heads repeated for
+    their query groups and an explicit causal mask."""
+    T, Hq, d = q.shape
+    L, Hkv, _ = k.shape
+    kk = torch.from_numpy(k).double().repeat_interleave(Hq // Hkv, dim=1).permute(1, 0, 2)  # [Hq, L, d]
+    vv = torch.from_numpy(v).double().repeat_interleave(Hq // Hkv, dim=1).permute(1, 0, 2)
+    qq = torch.from_numpy(q).double().permute(1, 0, 2)  # [Hq, T, d]
+    mask = torch.from_numpy(np.arange(L)[None, :] <= np.asarray(q_pos)[:, None])  # [T, L]
+    o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask)
+    return o.permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,L", [(1, 4, 1, 37), (3, 20, 5, 130), (16, 8, 2, 64)])
+def test_attention_matches_torch_sdpa(T, Hq, Hkv, L, attn_fn=None):
+    attn_fn = attn_fn or O.attention
+    rng = np.random.default_rng(T + L)
+    q, k, v = rng.standard_normal((T, Hq, 128)), rng.standard_normal((L, Hkv, 128)), rng.standard_normal((L, Hkv, 128))
+    q_pos = np.arange(L - T, L)
+    assert np.allclose(attn_fn(q, k, v, q_pos), _sdpa_reference(q, k, v, q_pos), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(4)
+    q, k, v = rng.standard_normal((1, 2, 128)), rng.standard_normal((5, 1, 128)), rng.standard_normal((5, 1, 128))
+    # a query at position 0 sees only key 0: the output is v_0
+    assert np.allclose(O.attention(q, k, v, np.array([0]))[0, :, :], np.repeat(v[0], 2, axis=0), rtol=0, atol=1e-15)
+    # identical keys: uniform weights, the mean of the visible values
+    kk = np.repeat(k[:1], 5, axis=0)
+    assert np.allclose(O.attention(q, kk, v, np.array([4]))[0, 0], v[:, 0].mean(axis=0), rtol=1e-13, atol=1e-15)
+
+
+def _attention_mutant(kind):
+    def attn(q, k, v, q_pos):
+        T, Hq, d = q.shape
+        L, Hkv, _ = k.shape
+        out = np.zeros((T, Hq, d))
+        for t in range(T):
+            n = L if kind == "not_causal" else int(q_pos[t]) + 1
+            for h in range(Hq):
+                kh = h % Hkv if kind == "heads_interleaved" else h // (Hq // Hkv)
+                s = (k[:n, kh] @ q[t, h]) / (d if kind == "scale_by_d" else math.sqrt(d))
+                w = np.exp(s - s.max())
+                out[t, h] = (w / w.sum()) @ v[:n, kh]
+        return out
+    return attn
+
+
+@pytest.mark.parametrize("kind", ["not_causal", "heads_interleaved", "scale_by_d"])
+def test_attention_pin_catches_planted_mistakes(kind):
+    with pytest.raises(AssertionError):
+        test_attention_matches_torch_sdpa(3, 20, 5, 130, attn_fn=_attention_mutant(kind))
+
+
+def test_rope_pin_catches_a_sign_flip(monkeypatch):
+    orig = O.apply_rope
+    monkeypatch.setattr(O, "apply_rope", lambda x, p, th: orig(x, -np.asarray(p, dtype=np.float64), th))
+    with pytest.raises(AssertionError):
+        test_rope_equals_complex_rotation()
