@@ -280,6 +280,36 @@ bitnet_status bitnet_decoder_block(const void* x, const void* attn_out, bitnet_d
                                    void* out_k, void* out_v, void* out_o, void* out_ffn,
                                    bitnet_dtype ot, void* ws, size_t ws_bytes, bitnet_stream s);
 
+/* The attention between a block's q/k/v and o projections at decode (the rest of the
+ * decoder block).  The BitNet pages keep the transformer's attention and only replace its
+ * linear layers ("Add BitNet" in flash-linear-attention: transformer code with nn.Linear
+ * swapped for BitLinear; [IQ1] the per-block attn_q/k/v/output tensors), so these compute the
+ * textbook form.  Head size d must be 128.
+ *
+ * bitnet_rope_kv_append: rotary embedding of q [T, Hq, d] and k [T, Hkv, d] (bf16 or fp32,
+ * the projections' outputs) at positions pos0 + t: for i < d/2 the pair (x_i, x_{i+d/2})
+ * turns by a = p theta^(-2i/d) (angle, sine and cosine in fp64, the rotation in fp32).  The
+ * rotated q goes to q_rot (fp32 [T, Hq, d]); the rotated k and the unchanged v are appended
+ * to the KV cache k_cache / v_cache (bf16 [Hkv][L_max][d], rows pos0 .. pos0 + T - 1, rounded
+ * to nearest even).  Errors: NULL, SHAPE (d != 128, Hq % Hkv, pos0 + T > L_max, theta <= 0),
+ * DTYPE. */
+bitnet_status bitnet_rope_kv_append(const void* q, const void* k, const void* v, bitnet_dtype xt, int64_t T,
+                                    int64_t Hq, int64_t Hkv, int64_t d, int64_t pos0, double theta, float* q_rot,
+                                    void* k_cache, void* v_cache, int64_t L_max, bitnet_stream s);
+
+/* Workspace of bitnet_attention_decode for L cache rows in use, in bytes (0 if invalid). */
+size_t bitnet_attention_workspace_bytes(int64_t T, int64_t Hq, int64_t Hkv, int64_t L);
+
+/* Causal grouped-query attention of T new tokens (positions pos0 .. pos0 + T - 1, already in
+ * the cache) against cache rows 0 .. pos0 + t: out[t, h] = softmax(q_rot[t, h] . k / sqrt(d)) v
+ * with key/value head h / (Hq / Hkv), in fp32 (split over 64-row chunks of the cache, merged
+ * exactly as running maxima and sums), written as bf16 or fp32 [T, Hq, d].  T * Hq / Hkv <= 128.
+ * ws: bitnet_attention_workspace_bytes(T, Hq, Hkv, pos0 + T) bytes, 16-byte aligned.
+ * Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
+bitnet_status bitnet_attention_decode(const float* q_rot, const void* k_cache, const void* v_cache, int64_t T,
+                                      int64_t Hq, int64_t Hkv, int64_t d, int64_t pos0, int64_t L_max, void* out,
+                                      bitnet_dtype ot, void* ws, size_t ws_bytes, bitnet_stream s);
+
 /* Synchronises `s`, then reads and clears the device status word of the current
  * device: BITNET_OK, or BITNET_ERR_TIMEOUT if a kernel gave up a bounded wait since
  * the last read. */

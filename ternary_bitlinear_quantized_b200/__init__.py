@@ -86,6 +86,11 @@ def lib() -> ctypes.CDLL:
         "bitnet_decoder_block": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
                                        c_i64, c_i64, c_i64, c_i64, c_i64, c_i, c_f, c_p, c_p, c_p, c_p, c_p, c_i,
                                        c_p, c_sz, c_p]),
+        "bitnet_rope_kv_append": (c_i, [c_p, c_p, c_p, c_i, c_i64, c_i64, c_i64, c_i64, c_i64, ctypes.c_double, c_p,
+                                        c_p, c_p, c_i64, c_p]),
+        "bitnet_attention_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64]),
+        "bitnet_attention_decode": (c_i, [c_p, c_p, c_p, c_i64, c_i64, c_i64, c_i64, c_i64, c_i64, c_p, c_i, c_p, c_sz,
+                                          c_p]),
         "bitnet_get_device_status": (c_i, [c_p]),
         "bitnet_debug_set_wait_limit": (c_i, [ctypes.c_longlong]),
         "bitnet_status_string": (ctypes.c_char_p, [c_i]),
@@ -355,6 +360,40 @@ def decoder_block(x, attn_out, gains: dict, packed: dict, NKV: int, I: int, act:
                                       _ptr(outs["ffn"]), _dtype_code(outs["ffn"].dtype), _ptr(ws), ws.numel(),
                                       _stream(stream)), "decoder_block")
     return outs
+
+
+def rope_kv_append(q, k, v, pos0: int, theta: float, k_cache, v_cache, q_rot=None, stream=None) -> torch.Tensor:
+    """Rotate q [T, Hq, 128] and k [T, Hkv, 128] at positions pos0 + t; append k (rotated) and v
+    to the bf16 caches [Hkv, L_max, 128].  Returns q_rot (fp32 [T, Hq, 128])."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, nm)
+    qr = q_rot if q_rot is not None else torch.empty(T, Hq, d, dtype=torch.float32, device=q.device)
+    _check(lib().bitnet_rope_kv_append(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), T, Hq, Hkv, d, pos0,
+                                       float(theta), _ptr(qr), _ptr(k_cache), _ptr(v_cache), k_cache.shape[1],
+                                       _stream(stream)), "rope_kv_append")
+    return qr
+
+
+def attention_workspace_bytes(T: int, Hq: int, Hkv: int, L: int) -> int:
+    return int(lib().bitnet_attention_workspace_bytes(T, Hq, Hkv, L))
+
+
+def attention_decode(q_rot, k_cache, v_cache, pos0: int, out_dtype=torch.bfloat16, out=None, ws=None,
+                     stream=None) -> torch.Tensor:
+    """Causal GQA attention of q_rot [T, Hq, 128] (positions pos0 + t) over cache rows 0..pos0 + t."""
+    T, Hq, d = q_rot.shape
+    Hkv, L_max = k_cache.shape[0], k_cache.shape[1]
+    for t, nm in ((q_rot, "q_rot"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, nm)
+    o = out if out is not None else torch.empty(T, Hq, d, dtype=out_dtype, device=q_rot.device)
+    nws = attention_workspace_bytes(T, Hq, Hkv, pos0 + T)
+    w = ws if ws is not None else torch.empty(max(nws, 16), dtype=torch.uint8, device=q_rot.device)
+    _check(lib().bitnet_attention_decode(_ptr(q_rot), _ptr(k_cache), _ptr(v_cache), T, Hq, Hkv, d, pos0, L_max,
+                                         _ptr(o), _dtype_code(o.dtype), _ptr(w), w.numel(), _stream(stream)),
+           "attention_decode")
+    return o
 
 
 def debug_set_wait_limit(cycles: int) -> None:

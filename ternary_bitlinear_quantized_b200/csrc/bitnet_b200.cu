@@ -15,6 +15,7 @@
 #include "engine.cuh"
 #include "gemm_tc.cuh"
 #include "shard.cuh"
+#include "attention.cuh"
 
 namespace bitnet {
 
@@ -113,20 +114,6 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2-D tensor of 32-bit words [rows, cols] (row stride `stride` bytes), box box_cols x box_rows.
-static bool make_map_u32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
-                         uint32_t box_cols, uint32_t box_rows) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {stride};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------ quant
@@ -267,31 +254,8 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
 }
 
 // ------------------------------------------------------------------ decode engine plans
-constexpr int ENG_SLOT_MAX = 40 * 1024;       // bytes of one ring slot at most
+constexpr int ENG_RING_MAX = 160 * 1024;      // bytes of weights in flight per SM at most
 constexpr int ENG_LOCAL_MAX_TK = 16 * 1024;   // T * K up to which every CTA quantises for itself
-constexpr int ENG_QS_GLOBAL_MAX = 32 * 1024;  // given activations up to this size are staged in shared memory
-
-// Stage geometry of one GEMV phase: K-chunks of C 32-bit words with C = 16 (mod 32) (a
-// consumer step is 16 words, and the rows of a 16-row box are then 64 (mod 128) bytes apart,
-// so two adjacent rows fall in different halves of the shared-memory banks), C <= 240 (the
-// TMA box limit is 256 elements), and the stage (tensors x 16 rows x C words) within
-// slot_max bytes.  The last chunk of a row may be partly outside the tensor (zero-filled).
-static void eng_chunks(EngPhase& p, int slot_max) {
-  const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-  const int W = p.K / 16;
-  int C = 16;
-  for (int n = 1; n <= W; ++n) {
-    int c = (W + n - 1) / n;
-    c = c <= 16 ? 16 : (c - 16 + 31) / 32 * 32 + 16;
-    if (c <= 240 && NT * 64 * c <= slot_max) {
-      C = c;
-      break;
-    }
-  }
-  p.chunk_words = C;
-  p.n_chunks = (W + C - 1) / C;
-  p.stage_bytes = NT * 64 * C;
-}
 
 static EngPhase eng_gemv(int K, bool ffn, int n_tensors, const uint8_t* const* packed, const int64_t* N,
                          void* const* out, int32_t* const* dbg, int out_dtype, int act, float* h) {
@@ -353,6 +317,20 @@ static EngPhase eng_quant(const void* x, int x_f32, int K, const float* gain, in
 static bool eng_local_ok(int64_t T, int64_t K) { return T * K <= ENG_LOCAL_MAX_TK && K <= ENG_REG_MAX_K; }
 static bool eng_quant_ok(int64_t K) { return K <= ENG_LOCAL_MAX_K; }
 
+// Tensor map of an I2_S tensor [N, K] as 8-byte elements [N, K/32], box CB/8 x 16 rows
+// (chunked stages of the decode engine).
+static bool make_map_u64(CUtensorMap* m, const void* base, uint64_t N, uint64_t K, uint32_t CB) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {K / 32, N};
+  const cuuint64_t strides[1] = {K / 4};
+  const cuuint32_t box[2] = {CB / 8, (cuuint32_t)GEMV_ROWS};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_INT64, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch the engine over the phases in `a` (a.T, a.eps, a.n_phases, a.ph, a.counters set).
 static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   static_assert(sizeof(EngArgs) % 16 == 0, "EngArgs is copied with 16-byte loads");
@@ -363,19 +341,27 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
     if (ph_is_gemv(a.ph[i].kind) && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
   const int gmax = sms < ENG_MAX_GRID ? sms : ENG_MAX_GRID;  // per-CTA partials are sized for ENG_MAX_GRID
   const int grid = multi ? gmax : (max_tiles < gmax ? max_tiles : gmax);
-  int acc_ints = 0, qs = 0, xs = 0;
+  int acc_ints = 0, qs = 0, xs = 0, slot = 0;
+  EngMaps maps;
+  memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < a.n_phases; ++i) {
-    const EngPhase& p = a.ph[i];
+    EngPhase& p = a.ph[i];
     if ((p.kind == PH_QUANT || (ph_is_gemv(p.kind) && p.src == SRC_LOCAL)) && p.K > ENG_REG_MAX_K && p.K > xs) xs = p.K;
     if (!ph_is_gemv(p.kind)) continue;
     const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
     const int per = (p.n_tiles + grid - 1) / grid * NT * GEMV_ROWS * a.T;
     if (per > acc_ints) acc_ints = per;
-    // Activations staged in shared memory: always for SRC_LOCAL; given ones when they fit
-    // and a CTA has at least three tiles to reuse them over (else the copy is only latency).
-    const int xp = (p.K + 255) / 256 * 256 + 64;
-    a.ph[i].xstage = p.src == SRC_GLOBAL && a.T * xp <= ENG_QS_GLOBAL_MAX && (p.n_tiles + grid - 1) / grid >= 3;
-    if ((p.src == SRC_LOCAL || a.ph[i].xstage) && a.T * xp > qs) qs = a.T * xp;
+    if (!eng_plan(p.K, a.T, ENG_SLOT_MAX, ENG_ACT_MAX, p.g))
+      return cuda_fail(cudaErrorInvalidConfiguration, "k_engine stage geometry");
+    if (p.src == SRC_LOCAL && !p.g.full_rows)  // local quantisation writes whole rows
+      return cuda_fail(cudaErrorInvalidConfiguration, "k_engine local activations");
+    if (a.T * p.g.x_pitch > qs) qs = a.T * p.g.x_pitch;
+    const int sb = (p.g.slot_bytes + 1023) / 1024 * 1024;  // TMA destinations 1024-byte aligned
+    if (sb > slot) slot = sb;
+    if (!p.g.full_rows)
+      for (int u = 0; u < p.n_tensors; ++u)
+        if (!make_map_u64(&maps.m[i][u], p.t[u].packed, (uint64_t)p.t[u].N, (uint64_t)p.K, (uint32_t)p.g.CB))
+          return cuda_fail(cudaErrorInvalidValue, "tensor map (engine weights)");
   }
   qs = (qs + 127) / 128 * 128;
   acc_ints = (acc_ints + 3) / 4 * 4;
@@ -388,27 +374,11 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   cudaGetDevice(&dev);
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int budget = max_optin - (int)fa.sharedSizeBytes - 1024 - 256;  // 1024: ring alignment
-  // Slots: about six fit, at most ENG_SLOT_MAX bytes each (larger TMA boxes stream faster
-  // than more, smaller ones).
+  const int budget = max_optin - (int)fa.sharedSizeBytes - 1024;  // 1024: ring alignment
   const int ring = budget - acc_ints * 4 - qs - xs * 4;
-  int slot_max = ring / 6 - 16;
-  if (slot_max > ENG_SLOT_MAX) slot_max = ENG_SLOT_MAX;
-  int slot = 0;
-  EngMaps maps;
-  memset(&maps, 0, sizeof(maps));
-  for (int i = 0; i < a.n_phases; ++i) {
-    EngPhase& p = a.ph[i];
-    if (!ph_is_gemv(p.kind)) continue;
-    eng_chunks(p, slot_max);
-    if (p.stage_bytes > slot) slot = p.stage_bytes;
-    for (int u = 0; u < p.n_tensors; ++u)
-      if (!make_map_u32(&maps.m[i][u], p.t[u].packed, (uint64_t)(p.K / 16), (uint64_t)p.t[u].N, (uint64_t)(p.K / 4),
-                        (uint32_t)p.chunk_words, (uint32_t)GEMV_ROWS))
-        return cuda_fail(cudaErrorInvalidValue, "tensor map (engine weights)");
-  }
-  slot = (slot + 127) / 128 * 128;
+  if (slot == 0) slot = 1024;  // no product phase (not planned by this library, but harmless)
   int slots = ring / (slot + 16);
+  if (slots * slot > ENG_RING_MAX) slots = ENG_RING_MAX / slot;
   if (slots > ENG_MAX_SLOTS) slots = ENG_MAX_SLOTS;
   if (slots < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_engine shared memory");
   a.n_slots = slots;
@@ -419,6 +389,11 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4;
   e = opt_in_smem((const void*)kern, 6 + tg - 1);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attribute");
+  // Grid barriers need every CTA resident at once: one CTA per SM must fit.
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ENG_THREADS, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "k_engine occupancy");
+  if (per_sm < 1 || grid > per_sm * sms) return cuda_fail(cudaErrorCooperativeLaunchTooLarge, "k_engine residency");
   e = launch(kern, dim3(grid), dim3(ENG_THREADS), smem, s, true, a, maps);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine");
   return BITNET_OK;
@@ -698,6 +673,76 @@ bitnet_status bitnet_dequant_acc(const int32_t* acc, const float* s_x, const uin
                          reinterpret_cast<cudaStream_t>(stream), true, acc, s_x, beta, (long long)T, (int)N, out,
                          (int)ot);
   return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_dequant_acc");
+}
+
+// ---------------------------------------------------------------- attention (decode)
+bitnet_status bitnet_rope_kv_append(const void* q, const void* k, const void* v, bitnet_dtype xt, int64_t T, int64_t Hq,
+                                    int64_t Hkv, int64_t d, int64_t pos0, double theta, float* q_rot, void* k_cache,
+                                    void* v_cache, int64_t L_max, bitnet_stream stream) {
+  if (xt != BITNET_BF16 && xt != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (T < 0 || T > 0x7FFFFFFFll || d != ATT_D || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Hq > 4096 || pos0 < 0 ||
+      L_max <= 0 || pos0 + T > L_max || !(theta > 0.0))
+    return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!q || !k || !v || !q_rot || !k_cache || !v_cache) return BITNET_ERR_NULL;
+  const long long total = T * (Hq + 2 * Hkv) * (ATT_D / 2);
+  const long long want = (total + 255) / 256, cap = (long long)device_sm_count() * 16;
+  const dim3 grid((unsigned)(want < cap ? want : cap));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (xt == BITNET_BF16)
+    e = launch(k_rope_append<__nv_bfloat16>, grid, dim3(256), 0, s, true, reinterpret_cast<const __nv_bfloat16*>(q),
+               reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), (int)T, (int)Hq,
+               (int)Hkv, (long long)pos0, theta, q_rot, reinterpret_cast<__nv_bfloat16*>(k_cache),
+               reinterpret_cast<__nv_bfloat16*>(v_cache), (long long)L_max);
+  else
+    e = launch(k_rope_append<float>, grid, dim3(256), 0, s, true, reinterpret_cast<const float*>(q),
+               reinterpret_cast<const float*>(k), reinterpret_cast<const float*>(v), (int)T, (int)Hq, (int)Hkv,
+               (long long)pos0, theta, q_rot, reinterpret_cast<__nv_bfloat16*>(k_cache),
+               reinterpret_cast<__nv_bfloat16*>(v_cache), (long long)L_max);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_rope_append");
+}
+
+size_t bitnet_attention_workspace_bytes(int64_t T, int64_t Hq, int64_t Hkv, int64_t L) {
+  if (T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0) return 0;
+  const long long chunks = (L + ATT_CHUNK - 1) / ATT_CHUNK;
+  return (size_t)chunks * Hkv * (T * (Hq / Hkv)) * (ATT_D + 2) * sizeof(float);
+}
+
+bitnet_status bitnet_attention_decode(const float* q_rot, const void* k_cache, const void* v_cache, int64_t T,
+                                      int64_t Hq, int64_t Hkv, int64_t d, int64_t pos0, int64_t L_max, void* out,
+                                      bitnet_dtype ot, void* ws, size_t ws_bytes, bitnet_stream stream) {
+  if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
+  if (T < 0 || d != ATT_D || Hq <= 0 || Hkv <= 0 || Hq % Hkv || pos0 < 0 || L_max <= 0 || pos0 + T > L_max ||
+      T * (Hq / Hkv) > ATT_MAX_ROWS || Hq > 4096 || (pos0 + T + ATT_CHUNK - 1) / ATT_CHUNK > 65535)
+    return BITNET_ERR_SHAPE;
+  if (T == 0) return BITNET_OK;
+  if (!q_rot || !k_cache || !v_cache || !out) return BITNET_ERR_NULL;
+  if (!aligned16(q_rot) || !aligned16(k_cache) || !aligned16(v_cache)) return BITNET_ERR_ALIGN;
+  if (!ws || ws_bytes < bitnet_attention_workspace_bytes(T, Hq, Hkv, pos0 + T)) return BITNET_ERR_WORKSPACE;
+  if (!aligned16(ws)) return BITNET_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int R = (int)(T * (Hq / Hkv));
+  const int chunks = (int)((pos0 + T + ATT_CHUNK - 1) / ATT_CHUNK);
+  const size_t smem = attn_partial_smem(R);
+  static std::atomic<int> attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_done[dev & 63].load(std::memory_order_acquire)) {
+    cudaError_t ea = cudaFuncSetAttribute(k_attn_partial, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)attn_partial_smem(ATT_MAX_ROWS));
+    if (ea != cudaSuccess) return cuda_fail(ea, "k_attn_partial attribute");
+    attr_done[dev & 63].store(1, std::memory_order_release);
+  }
+  float* part = reinterpret_cast<float*>(ws);
+  cudaError_t e = launch(k_attn_partial, dim3((unsigned)chunks, (unsigned)Hkv), dim3(ATT_THREADS), smem, s, true,
+                         q_rot, reinterpret_cast<const __nv_bfloat16*>(k_cache),
+                         reinterpret_cast<const __nv_bfloat16*>(v_cache), (int)T, (int)Hq, (int)Hkv, (long long)pos0,
+                         (long long)L_max, part);
+  if (e != cudaSuccess) return cuda_fail(e, "k_attn_partial");
+  e = launch(k_attn_combine, dim3((unsigned)(T * Hq)), dim3(ATT_D), 0, s, true, (const float*)part, (int)T, (int)Hq,
+             (int)Hkv, chunks, out, (int)ot);
+  return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "k_attn_combine");
 }
 
 static size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }

@@ -17,11 +17,14 @@
 // is being completed) fills the wait.
 //
 // Weights do not depend on any phase, so a producer warp streams the packed bytes of
-// ALL phases of this CTA, in phase order, through a ring of shared-memory slots with 2-D
-// TMA boxes; it starts before griddepcontrol.wait, i.e. while the previous kernel on the
-// stream is still running.  The 15 consumer warps work in groups, each group owning a
-// 16-row tile over all of its K-chunks (one AND per 2-bit field, mma.sync m16n8k32
-// u8 x s8, per-field accumulators combined exactly once per tile).
+// ALL phases of this CTA, in phase order, through a ring of shared-memory slots; it starts
+// before griddepcontrol.wait, i.e. while the previous kernel on the stream is still running.
+// A slot holds one tensor's weights: whole 16-row tiles fetched as one contiguous 1-D bulk
+// copy (rows of up to 2 KB), or one 16-row x 2 KB 2-D TMA box of longer rows (geometry in
+// engine_sched.h).  All 15 consumer warps work on every slot, taking its 64-byte steps in
+// turn (one AND per 2-bit field, mma.sync m16n8k32 u8 x s8, per-field accumulators combined
+// exactly once per tile and added into the tile's shared accumulator).  The steps are dealt
+// to the warps round-robin, continuing from stage to stage, so the warps' loads even out.
 //
 // Arithmetic and sources as in quant.cuh ("Add optional RMSNorm support to BitNet
 // quantization": BitNetRMSNorm before quantisation) and gemv.cuh ("fix: I2_S ARM kernel
@@ -40,7 +43,7 @@
 
 namespace bitnet {
 
-constexpr int ENG_CONS_WARPS = 15;  // + 1 producer warp = 16 warps, 4 per SM sub-partition
+constexpr int ENG_CONS_WARPS = 15;  // + 1 producer warp: 16 warps, 4 per SM sub-partition (128 registers each)
 constexpr int ENG_CONS = ENG_CONS_WARPS * 32;
 constexpr int ENG_THREADS = ENG_CONS + 32;
 constexpr int ENG_MAX_PHASES = 8;
@@ -81,14 +84,11 @@ struct EngPhase {
   float* pmax;
   long long* psum;
   int bar_a, bar_b;
-  int xstage;  // SRC_GLOBAL: copy the activations into shared memory first (else read in place)
-  // Stage geometry: a stage is one 2-D TMA box per tensor of 16 rows (one tile) x
-  // chunk_words 32-bit words (a K-chunk; chunk_words = 16 mod 32, so the rows of a box are
-  // 64 mod 128 bytes apart); stage_bytes = tensors x 64 x chunk_words.
-  int chunk_words, n_chunks, stage_bytes;
+  EngGeom g;  // stage geometry of a product phase (engine_sched.h)
 };
 
-// One tensor map per tensor and phase: the packed rows viewed as [N, K/16] 32-bit words.
+// One tensor map per tensor and phase (chunked mode): the packed rows viewed as
+// [N, K/32] 8-byte elements, box CB/8 x 16.
 struct alignas(64) EngMaps {
   CUtensorMap m[ENG_MAX_PHASES][4];
 };
@@ -531,154 +531,92 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
   return true;
 }
 
-// ------------------------------------------------------------------ stage schedule
-// EngSched / EngOwnStages (engine_sched.h): the producer walks the whole sequence, each
-// consumer group only its own stages.
-
-// Wait until the producer has tagged ring slot `tag` with stage `want` (bounded, like the
-// barrier waits).
-BN_DEV bool wait_slot_tag(const volatile int* tag, int want) {
-  if (*tag == want) return true;
-  const long long t0 = clock64(), lim = c_wait_limit;
-  while (*tag != want) {
-    if (clock64() - t0 > lim) {
-      atomicExch(&g_device_status, (int)BITNET_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-
-// ------------------------------------------------------------------ products of one phase
-// The consumer warp's part of one GEMV phase: walk the stage sequence (advancing the ring
-// position `slot`/`par` for every stage), and for the stages of its group wait for the
-// data, run its share of the 64-byte steps, release the slot, and after the last chunk of
-// a unit add its partial sums to the tile's shared accumulator acc[tile][u][row][token].
-// Lane (gid, r) holds rows gid and gid + 8 of the tile, bytes 16 r .. 16 r + 15 of each
-// step (the A fragments of mma.sync m16n8k32, one AND per 2-bit field), and the
-// activations of tokens gid (and 8 + gid), or of token T - 1 where those do not exist.
-// XSM: activations in shared memory (layout eng_perm, lane addresses xs_a / xs_b); else in
-// global memory in plain order (xg_a / xg_b).  Returns false if a wait gave up.
-template <int TG, int NT, bool XSM>
-__device__ __forceinline__ bool eng_phase_products(const EngArgs& a, const EngPhase& p, int nt, uint32_t ring_s,
-                                                   uint32_t bar0, const volatile int* slot_tag, int& seq,
-                                                   int& slot, uint32_t& par, int* acc, uint32_t xs_a,
-                                                   uint32_t xs_b, const int8_t* xg_a, const int8_t* xg_b) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, r = lane & 3;
-  const int T = a.T;
-  const int ng = eng_groups(nt), gw = ENG_CONS_WARPS / ng;
-  const int my_grp = warp / gw, my_i = warp - my_grp * gw;
-  const int C = p.chunk_words, W = p.K >> 4, pitch = 4 * C;
-  int f[NT][TG][4][4];
-#pragma unroll
-  for (int u = 0; u < NT; ++u)
+// ------------------------------------------------------------------ products of one stage
+// Partial sums of one tile of one tensor, per 2-bit field: f[tg][g][i] is the mma
+// accumulator of token group tg (tokens 8 tg + ..) and field g (codes scaled by 4^(3-g)).
+template <int TG>
+struct EngAcc {
+  int f[TG][4][4];
+  BN_DEV void zero() {
 #pragma unroll
     for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
       for (int g = 0; g < 4; ++g)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) f[u][tg][g][i] = 0;
-  // This group's stages in sequence order; `done` is how far the ring position (slot, par)
-  // has been advanced.
-  const EngSched sc(nt, p.n_chunks);
-  EngOwnStages own(sc, my_grp);
-  int rot = 0, done = 0;
-  int pos, tl, c;
-  bool last;
-  while (own.next(pos, tl, c, last)) {
-    // advance the ring position to stage `pos`
-    slot += pos - done;
-    done = pos + 1;
-    while (slot >= a.n_slots) {
-      slot -= a.n_slots;
-      par ^= 1u;
-    }
-    const int s = slot;
-    const uint32_t ph = par;
-    if (++slot == a.n_slots) {
-      slot = 0;
-      par ^= 1u;
-    }
-    // Groups run ahead of one another, so the slot's previous fill may still be in flight;
-    // a parity wait is only unambiguous once the producer has taken the slot for this stage.
-    if (!wait_slot_tag(slot_tag + s, seq + pos)) return false;
-    if (!mbar_wait_bounded(bar0 + 8u * s, ph)) return false;
-    const int cbytes = 4 * min(C, W - c * C);  // bytes of the rows inside the tensor
-    const int nsteps = (cbytes + 63) >> 6;
-    int t = my_i - rot;  // the group's warps take the steps in turn, starting one later each stage
-    if (t < 0) t += gw;
-    if (++rot == gw) rot = 0;
-    const uint32_t wbase = ring_s + s * a.slot_bytes + gid * pitch + 16 * r;
-    const int gs0 = c * (C >> 4);  // 64-byte step index of the chunk's first step
-    for (; t < nsteps; t += gw) {
-      uint4 wa[NT], wb[NT];
+        for (int i = 0; i < 4; ++i) f[tg][g][i] = 0;
+  }
+  // Combine the fields exactly (field g's sums are multiples of 4^(3-g)) and add this warp's
+  // share into the tile's shared accumulator at[row * T + tok]; then restart.
+  BN_DEV void flush(int* at, int T, int gid, int r) {
 #pragma unroll
-      for (int u = 0; u < NT; ++u) {
-        wa[u] = lds128(wbase + u * 16 * pitch + 64 * t);
-        wb[u] = lds128(wbase + u * 16 * pitch + 8 * pitch + 64 * t);
-      }
-      // Lanes of tokens >= T read another token's activations: they only feed accumulator
-      // columns that are never used.
-      uint4 xa[4], xb[4];
-      if (XSM) {
-        const uint32_t xo = 256u * (gs0 + t);
+    for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          xa[g] = lds128(xs_a + xo + 64 * g);
-          if (TG > 1) xb[g] = lds128(xs_b + xo + 64 * g);
-        }
-      } else {
-        // Weight bytes past the row end are zero (TMA fill); the activations there lie past
-        // the row in global memory, so those lanes read the row's first bytes instead.
-        const long long xo = 64 * t + 16 * r < cbytes ? 256LL * (gs0 + t) : 0;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          xa[g] = *reinterpret_cast<const uint4*>(xg_a + xo + 32 * g);
-          if (TG > 1) xb[g] = *reinterpret_cast<const uint4*>(xg_b + xo + 32 * g);
+      for (int i = 0; i < 4; ++i) {
+        const int tok = tg * 8 + 2 * r + (i & 1);
+        if (tok < T) {
+          const int v = (f[tg][0][i] >> 6) + (f[tg][1][i] >> 4) + (f[tg][2][i] >> 2) + f[tg][3][i];
+          atomicAdd(at + (gid + ((i & 2) ? 8 : 0)) * T + tok, v);
         }
       }
+    zero();
+  }
+};
+
+// This warp's 64-byte steps of one 16-row tile in a stage: steps t = t0, t0 + 15, .. < S.
+// Lane (gid, r) holds rows gid and gid + 8 of the tile, bytes 16 r .. 16 r + 15 of each step
+// (the A fragments of mma.sync m16n8k32, one AND per 2-bit field), and the activations of
+// tokens gid (and 8 + gid) -- token T - 1 where those do not exist; those lanes only feed
+// accumulator columns that are never used.  wrow: shared address of row gid's step 0 at
+// byte 16 r; P: row pitch; xa / xb: shared address of the tokens' step 0 (+ 16 r).
+template <int TG>
+BN_DEV void eng_tile_steps(EngAcc<TG>& A, uint32_t wrow, int P, uint32_t xa_s, uint32_t xb_s, int t0, int S) {
+  for (int t = t0; t < S; t += ENG_CONS_WARPS) {
+    const uint4 wa = lds128(wrow + 64 * t), wb = lds128(wrow + 8 * P + 64 * t);
+    const uint32_t xo = 256u * t;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t m = 0x03030303u << (6 - 2 * g);
-#pragma unroll
-        for (int u = 0; u < NT; ++u) {
-          const uint32_t a0 = wa[u].x & m, a1 = wb[u].x & m, a2 = wa[u].y & m, a3 = wb[u].y & m;
-          const uint32_t a4 = wa[u].z & m, a5 = wb[u].z & m, a6 = wa[u].w & m, a7 = wb[u].w & m;
-          mma_u8s8(f[u][0][g], a0, a1, a2, a3, xa[g].x, xa[g].y);
-          mma_u8s8(f[u][0][g], a4, a5, a6, a7, xa[g].z, xa[g].w);
-          if (TG > 1) {
-            mma_u8s8(f[u][TG - 1][g], a0, a1, a2, a3, xb[g].x, xb[g].y);
-            mma_u8s8(f[u][TG - 1][g], a4, a5, a6, a7, xb[g].z, xb[g].w);
-          }
-        }
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t m = 0x03030303u << (6 - 2 * g);
+      const uint32_t a0 = wa.x & m, a1 = wb.x & m, a2 = wa.y & m, a3 = wb.y & m;
+      const uint32_t a4 = wa.z & m, a5 = wb.z & m, a6 = wa.w & m, a7 = wb.w & m;
+      const uint4 x0 = lds128(xa_s + xo + 64 * g);
+      mma_u8s8(A.f[0][g], a0, a1, a2, a3, x0.x, x0.y);
+      mma_u8s8(A.f[0][g], a4, a5, a6, a7, x0.z, x0.w);
+      if (TG > 1) {
+        const uint4 x1 = lds128(xb_s + xo + 64 * g);
+        mma_u8s8(A.f[TG - 1][g], a0, a1, a2, a3, x1.x, x1.y);
+        mma_u8s8(A.f[TG - 1][g], a4, a5, a6, a7, x1.z, x1.w);
       }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive_count(bar0 + 8u * (a.n_slots + s), (uint32_t)ng);
-    if (last) {
-      int* at = acc + tl * NT * GEMV_ROWS * T;
-#pragma unroll
-      for (int u = 0; u < NT; ++u)
-#pragma unroll
-        for (int tg = 0; tg < TG; ++tg)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int v = (f[u][tg][0][i] >> 6) + (f[u][tg][1][i] >> 4) + (f[u][tg][2][i] >> 2) + f[u][tg][3][i];
-            const int row = gid + ((i & 2) ? 8 : 0), tok = tg * 8 + 2 * r + (i & 1);
-            if (tok < T) atomicAdd(at + (u * GEMV_ROWS + row) * T + tok, v);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) f[u][tg][g][i] = 0;
-          }
     }
   }
-  // past the phase's last stage
-  slot += sc.total() - done;
-  seq += sc.total();
-  while (slot >= a.n_slots) {
-    slot -= a.n_slots;
-    par ^= 1u;
+}
+
+// Stage activations [k0, k1) of all T tokens from global memory (plain int8 [T, K]) into
+// shared memory in the eng_perm layout, zero-padded to whole 256-in-feature steps.  The
+// rows were written by this launch's QUANT / SUBNORM phase or by the previous kernel: read
+// past L1.  Four 16-byte loads in flight per thread.
+BN_DEV void eng_stage_acts(const int8_t* q, int K, int T, int k0, int k1, int8_t* qs, int x_pitch) {
+  const int n16 = (k1 - k0) >> 4, padded = ((k1 - k0 + 255) & ~255) >> 4;
+  const int total = T * padded;
+  for (int base = threadIdx.x; base < total; base += 4 * ENG_CONS) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = base + j * ENG_CONS;
+      v[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < total) {
+        const int t = i / padded, u = i - t * padded;
+        if (u < n16) v[j] = __ldcg(reinterpret_cast<const uint4*>(q + (long long)t * K + k0 + 16 * u));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = base + j * ENG_CONS;
+      if (i < total) {
+        const int t = i / padded, u = i - t * padded;
+        *reinterpret_cast<uint4*>(qs + t * x_pitch + eng_perm(16 * u)) = v[j];
+      }
+    }
   }
-  return true;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -702,9 +640,9 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   __shared__ float s_loc_s[ENG_MAX_T];
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
   __shared__ float s_beta[ENG_MAX_PHASES][4];
-  volatile __shared__ int s_slot_tag[ENG_MAX_SLOTS];  // stage index the producer last put in each slot
   __shared__ SubScratch s_sub;
   __shared__ unsigned s_hmax[ENG_MAX_T];  // max |h| of this CTA's rows (gate/up epilogue)
+  __shared__ int s_issued;                // stages the producer issued (for the drain on exit)
 
   // TMA boxes land 1024-byte aligned.
   uint8_t* ring = smem + ((1024u - (smem_addr(smem) & 1023u)) & 1023u);
@@ -721,10 +659,10 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.n_slots; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), ENG_CONS_WARPS);  // each warp of the owning group arrives with count ng
-      s_slot_tag[s] = -1;
+      mbar_init(empty(s), ENG_CONS_WARPS);
     }
     s_abort = 0;
+    s_issued = 0;
     fence_mbar_init();
   }
   if (threadIdx.x < ENG_MAX_PHASES * 4) {  // per-tensor scales (weights: no dependency wait needed)
@@ -753,41 +691,73 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
 
   if (warp == ENG_CONS_WARPS) {
     // ------------------------------------------------------------ producer
-    // Lane u < NT issues the box of tensor u of each stage (no multicast).
-    int slot = 0, seq = 0;
+    // Walks the stage order of every product phase (engine_sched.h).  Lane 0 waits for the
+    // slot, sets the expected bytes and issues the copies (no multicast).
+    int slot = 0, issued = 0;
     uint32_t par = 0;
-    for (int pi = 0; pi < a.n_phases && !s_abort; ++pi) {
+    bool go = true;  // warp-uniform: false once a wait gave up or the consumers aborted
+    for (int pi = 0; pi < a.n_phases && go; ++pi) {
       const EngPhase& p = a.ph[pi];
       if (!ph_is_gemv(p.kind)) continue;
+      const EngGeom& G = p.g;
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
-      const uint32_t box_bytes = 64u * (uint32_t)p.chunk_words;
       int tb, te;
       tile_range(p, tb, te);
-      EngSched sc(te - tb, p.n_chunks);
-      int grp, tl, c;
-      bool last;
-      while (!s_abort && sc.next(grp, tl, c, last)) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_bounded(empty(slot), par ^ 1u);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          s_abort = 1;
-          break;
-        }
-        int ti, n0, nr;
-        locate(p, tb + tl, ti, n0, nr);
-        if (lane == 0) {
-          s_slot_tag[slot] = seq;
-          mbar_arrive_expect_tx(full(slot), (uint32_t)p.stage_bytes);
-        }
-        __syncwarp();
-        if (lane < NT)
-          tma_load_2d(smem_addr(ring + slot * a.slot_bytes + lane * box_bytes), &maps.m[pi][NT == 2 ? lane : ti],
-                      c * p.chunk_words, n0, full(slot));
-        ++seq;
-        if (++slot == a.n_slots) {
-          slot = 0;
-          par ^= 1u;
+      const int nt = te - tb;
+      for (int ac = 0; ac < G.n_ac && go; ++ac) {
+        const int wc0 = ac * G.ac_chunks, wc1 = min(G.n_chunks, wc0 + G.ac_chunks);
+        for (int tg0 = 0; tg0 < nt && go; tg0 += G.rs) {
+          const int ntg = min(G.rs, nt - tg0);
+          for (int u = 0; u < NT && go; ++u) {
+            for (int wc = wc0; wc < wc1 && go; ++wc) {
+              bool ok = true;
+              if (lane == 0) {
+                ok = s_abort == 0 && mbar_wait_bounded(empty(slot), par ^ 1u);
+                if (ok) {
+                  const uint32_t dst = smem_addr(ring + slot * a.slot_bytes);
+                  if (G.full_rows) {
+                    // runs of consecutive tiles of the same tensor: one contiguous copy each
+                    uint32_t bytes = 0;
+                    for (int pass = 0; pass < 2; ++pass) {
+                      if (pass == 1) mbar_arrive_expect_tx(full(slot), bytes);
+                      for (int i = 0; i < ntg;) {
+                        int ti, n0, nr;
+                        locate(p, tb + tg0 + i, ti, n0, nr);
+                        int j = i + 1, rows = nr;
+                        while (j < ntg) {
+                          int tj, m0, mr;
+                          locate(p, tb + tg0 + j, tj, m0, mr);
+                          if (tj != ti) break;
+                          rows += mr;
+                          ++j;
+                        }
+                        if (pass == 0) {
+                          bytes += (uint32_t)rows * G.RB;
+                        } else {
+                          const uint8_t* src = p.t[NT == 2 ? u : ti].packed + (long long)n0 * G.RB;
+                          bulk_g2s(dst + (uint32_t)(i * GEMV_ROWS * G.RB), src, (uint32_t)rows * G.RB, full(slot));
+                        }
+                        i = j;
+                      }
+                    }
+                  } else {
+                    int ti, n0, nr;
+                    locate(p, tb + tg0, ti, n0, nr);
+                    mbar_arrive_expect_tx(full(slot), (uint32_t)(GEMV_ROWS * G.CB));
+                    tma_load_2d(dst, &maps.m[pi][NT == 2 ? u : ti], wc * (G.CB >> 3), n0, full(slot));
+                  }
+                  s_issued = ++issued;
+                } else {
+                  s_abort = 1;
+                }
+              }
+              go = __shfl_sync(0xffffffffu, ok, 0);
+              if (++slot == a.n_slots) {
+                slot = 0;
+                par ^= 1u;
+              }
+            }
+          }
         }
       }
     }
@@ -798,7 +768,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     pdl_wait();  // activations and workspace belong to the previous kernel until now
     int slot = 0;       // ring position of the next stage
     uint32_t par = 0;   // and the phase parity of its barriers
-    int seq = 0;        // index of the phase's first stage in the producer's sequence
+    int rot = 0;        // round-robin position of the 64-byte steps over the warps
     // The SUBNORM phases accumulate sum_q with atomics: clear it before any CTA can get
     // there (the grid barrier of the gate/up phase comes first).
     if (blockIdx.x == 0 && threadIdx.x < T)
@@ -834,59 +804,94 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         grid_arrive(a.counters + p.arrive_barrier);
         continue;
       }
+      const EngGeom& G = p.g;
       const int NT = p.kind == PH_GEMV_FFN ? 2 : 1;
       int tb, te;
       tile_range(p, tb, te);
       const int nt = te - tb;
-      const int xp = eng_x_pitch(p.K), K16 = p.K >> 4;
-      // Activations of this phase: in shared memory (layout eng_perm) when they fit, else
-      // read in plain order from global memory.
       const bool local = p.src == SRC_LOCAL;
-      const bool xsm = local || p.xstage;
       if (local) {
+        // Quantise the raw activations in this CTA (whole row, full-row geometry), straight
+        // into the shared layout; zero the padding of the last 256-in-feature step.
         for (int t = 0; t < T; ++t) {
           quant_row(reinterpret_cast<const uint8_t*>(p.x) + (long long)t * p.K * (p.x_f32 ? 4 : 2), p.x_f32, p.K,
-                    p.gain, a.eps, qs + t * xp, true, s_loc_s + t, s_loc_sq + t, s_red, xs);
+                    p.gain, a.eps, qs + t * G.x_pitch, true, s_loc_s + t, s_loc_sq + t, s_red, xs);
+        }
+        const int pad16 = (((p.K + 255) & ~255) - p.K) >> 4;
+        for (int i = threadIdx.x; i < T * pad16; i += ENG_CONS) {
+          const int t = i / pad16, u = p.K / 16 + (i - t * pad16);
+          *reinterpret_cast<uint4*>(qs + t * G.x_pitch + eng_perm(16 * u)) = make_uint4(0u, 0u, 0u, 0u);
         }
         if (blockIdx.x == 0 && p.q != nullptr) {  // one plain-order copy for callers that read the intermediates
+          const int K16 = p.K >> 4;
           for (int i = threadIdx.x; i < T * K16; i += ENG_CONS) {
             const int t = i / K16, k = (i - t * K16) * 16;
             *reinterpret_cast<uint4*>(p.q + (long long)t * p.K + k) =
-                *reinterpret_cast<const uint4*>(qs + t * xp + eng_perm(k));
+                *reinterpret_cast<const uint4*>(qs + t * G.x_pitch + eng_perm(k));
           }
           if (threadIdx.x < T) {
             p.s[threadIdx.x] = s_loc_s[threadIdx.x];
             p.sq[threadIdx.x] = s_loc_sq[threadIdx.x];
           }
         }
-      } else if (xsm) {
-        // Written by this launch's QUANT phase or by the previous kernel: read past L1.
-        for (int i = threadIdx.x; i < T * K16; i += ENG_CONS) {
-          const int t = i / K16, k = (i - t * K16) * 16;
-          *reinterpret_cast<uint4*>(qs + t * xp + eng_perm(k)) =
-              __ldcg(reinterpret_cast<const uint4*>(p.q + (long long)t * p.K + k));
-        }
       }
       for (int i = threadIdx.x; i < nt * NT * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
       if (threadIdx.x < T) s_hmax[threadIdx.x] = 0u;
-      cons_sync();
 
       {
         const uint32_t qs_s = smem_addr(qs);
         const int ta = min(t_a, T - 1), tb2 = min(t_b, T - 1);
-        const uint32_t xs_a = qs_s + ta * xp + 16 * r, xs_b = qs_s + tb2 * xp + 16 * r;
-        const int8_t* xg_a = p.q + (long long)ta * p.K + 128 * (r >> 1) + 16 * (r & 1);
-        const int8_t* xg_b = p.q + (long long)tb2 * p.K + 128 * (r >> 1) + 16 * (r & 1);
+        const uint32_t xa0 = qs_s + ta * G.x_pitch + 16 * r, xb0 = qs_s + tb2 * G.x_pitch + 16 * r;
         const uint32_t ring_s = smem_addr(ring);
-#define ENG_PRODUCTS(NTV, XSMV)                                                                              \
-  eng_phase_products<TG, NTV, XSMV>(a, p, nt, ring_s, bar0, s_slot_tag, seq, slot, par, acc, xs_a, xs_b, xg_a, \
-                                    xg_b)
-        bool ok;
-        if (NT == 2)
-          ok = xsm ? ENG_PRODUCTS(2, true) : ENG_PRODUCTS(2, false);
-        else
-          ok = xsm ? ENG_PRODUCTS(1, true) : ENG_PRODUCTS(1, false);
-#undef ENG_PRODUCTS
+        EngAcc<TG> A;
+        A.zero();
+        // A warp whose wait gives up stops waiting and computing but keeps walking the stage
+        // order, so that every consumer thread meets the same named barriers; the decision
+        // to leave is taken together at the next one (barrier.red.or).
+        bool ok = true;
+        for (int ac = 0; ac < G.n_ac; ++ac) {
+          const int wc0 = ac * G.ac_chunks, wc1 = min(G.n_chunks, wc0 + G.ac_chunks);
+          if (!local) {
+            // the previous chunk's readers are done, then stage this chunk
+            if (named_sync_or(1, ENG_CONS, !ok)) {
+              ok = false;
+              break;
+            }
+            eng_stage_acts(p.q, p.K, T, 4 * wc0 * G.CB, min(p.K, 4 * wc1 * G.CB), qs, G.x_pitch);
+          }
+          if (named_sync_or(1, ENG_CONS, !ok)) {
+            ok = false;
+            break;
+          }
+          for (int tg0 = 0; tg0 < nt; tg0 += G.rs) {
+            const int ntg = min(G.rs, nt - tg0);
+            for (int u = 0; u < NT; ++u) {
+              for (int wc = wc0; wc < wc1; ++wc) {
+                if (ok && !mbar_wait_bounded(full(slot), par)) ok = false;
+                if (ok) {
+                  const int cbytes = min(G.CB, G.RB - wc * G.CB);
+                  const int S = (cbytes + 63) >> 6;
+                  const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (G.CB >> 6));
+                  const uint32_t sbase = ring_s + slot * a.slot_bytes + gid * G.CB + 16 * r;
+                  for (int tl = 0; tl < ntg; ++tl) {
+                    int t0 = warp - rot;
+                    if (t0 < 0) t0 += ENG_CONS_WARPS;
+                    eng_tile_steps<TG>(A, sbase + tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S);
+                    rot += S;
+                    while (rot >= ENG_CONS_WARPS) rot -= ENG_CONS_WARPS;
+                    if (wc == wc1 - 1) A.flush(acc + ((tg0 + tl) * NT + u) * GEMV_ROWS * T, T, gid, r);
+                  }
+                  __syncwarp();
+                  if (lane == 0) mbar_arrive(empty(slot));
+                }
+                if (++slot == a.n_slots) {
+                  slot = 0;
+                  par ^= 1u;
+                }
+              }
+            }
+          }
+        }
         if (!ok) s_abort = 1;
       }
       if (named_sync_or(1, ENG_CONS, s_abort != 0)) break;
@@ -931,6 +936,13 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   }
 
   __syncthreads();
+  // After an abort, copies the producer issued may still be in flight into this CTA's shared
+  // memory: wait for every slot's last fill to land (fixed limit) before the CTA exits.
+  if (s_abort && threadIdx.x == 0) {
+    const int issued = s_issued;
+    for (int k = (issued > a.n_slots ? issued - a.n_slots : 0); k < issued; ++k)
+      mbar_drain(full(k % a.n_slots), (uint32_t)((k / a.n_slots) & 1));
+  }
   if (threadIdx.x == 0 && a.counters != nullptr) {
     // The last CTA out zeroes the barrier counters for the next launch.
     __threadfence();

@@ -1,13 +1,21 @@
-// Stage schedule of a decode-engine GEMV phase (see engine.cuh): which CTA-local tile and
-// K-chunk every stage of the weight ring holds, in the order the producer warp issues them,
-// and each consumer group's own stages in closed form.  No CUDA dependency, so the host
-// test of the schedule compiles it as plain C++.
+// Stage geometry of a decode-engine product phase (see engine.cuh), shared by the host
+// planner, the producer warp and the consumer warps.  No CUDA dependency, so the host test
+// compiles it as plain C++.
 //
-// A phase gives a CTA nt tiles (16 weight rows each) of nch K-chunks.  The consumer warps
-// form ng groups; a group owns a tile for all of its chunks.  Tiles are dealt to the
-// groups in rounds of ng (stage order: chunk-major within a round, group-minor); the
-// `left` tiles of a last, partial round are each split into s contiguous chunk ranges
-// (units), unit u going to group u, and their stages run step-major over the units.
+// A stage (one ring slot) holds weights of ONE tensor: `rs` 16-row tiles x `CB` bytes of each
+// row.  Two modes:
+//   full rows  (CB == RB, the whole row): the tiles' rows are one contiguous byte range of
+//              the I2_S tensor, fetched with one 1-D bulk copy per run of tiles of the same
+//              tensor (large contiguous copies stream at close to the HBM peak);
+//   chunked    (rs == 1, CB < RB): one 2-D TMA box of 16 rows x CB bytes (8-byte elements,
+//              zero fill past the row end) per stage, for rows too long for a slot or for
+//              activations too large to stage whole.
+// The activations of the phase are staged in shared memory in chunks of `ac_chunks` weight
+// chunks (the whole row in full-row mode).  Stage order on a CTA that owns tiles [0, nt):
+//   for ac < n_ac:  for tg0 = 0, rs, 2 rs, .. < nt:  for u < NT:  for wc in chunks of ac:
+// (NT = 2 for the FFN's gate/up pair, whose stages alternate gate and up; else 1).  The
+// consumers' partial sums of a tile persist over the chunks of one activation chunk and one
+// tensor and are flushed after its last chunk.
 #pragma once
 
 #if defined(__CUDACC__)
@@ -18,110 +26,76 @@
 
 namespace bitnet {
 
-ENG_HD int eng_groups(int nt) { return nt >= 5 ? 5 : (nt >= 3 ? 3 : 1); }
+constexpr int ENG_BOX_MAX_BYTES = 2048;     // a TMA box row: 256 elements of 8 bytes
+constexpr int ENG_SLOT_MAX = 40 * 1024 + 64;  // bytes of one ring slot at most (a stage + slack)
+constexpr int ENG_ACT_MAX = 72 * 1024;        // shared memory for the staged activations
+constexpr int ENG_STAGE_TARGET = 40 * 1024;  // full-row stages group tiles up to this size
+constexpr int ENG_MAX_RS = 8;                // tiles per full-row stage at most
 
-struct EngSched {
-  int nch, ng, R, s, units, maxlen;
-  int a, b, q;
-  bool rem;
-  ENG_HD EngSched(int nt, int nch_) : nch(nch_), a(0), b(0), q(0), rem(false) {
-    ng = eng_groups(nt);
-    R = nt / ng;
-    const int left = nt - R * ng;
-    s = left == 0 ? 1 : (nch >= 2 ? (ng / left < nch ? ng / left : nch) : 1);
-    units = left * s;
-    maxlen = (nch + s - 1) / s;
-  }
-  // Chunk range [cb, ce) of unit u of the last round.
-  ENG_HD int unit_begin(int u) const { return nch * (u % s) / s; }
-  ENG_HD int unit_end(int u) const { return nch * (u % s + 1) / s; }
-  // Stages of the whole phase.
-  ENG_HD int total() const {
-    int n = R * ng * nch;
-    for (int u = 0; u < units; ++u) n += unit_end(u) - unit_begin(u);
-    return n;
-  }
-  // Next stage: owning group, tile (local index), chunk, and whether it is the last chunk
-  // of the group's share of the tile.  False at the end.
-  ENG_HD bool next(int& grp, int& tile, int& c, bool& last) {
-    while (true) {
-      if (!rem) {
-        if (a >= R) {
-          rem = true;
-          a = 0;
-          q = 0;
-          continue;
-        }
-        grp = q;
-        tile = a * ng + q;
-        c = b;
-        last = b == nch - 1;
-        if (++q == ng) {
-          q = 0;
-          if (++b == nch) {
-            b = 0;
-            ++a;
-          }
-        }
-        return true;
-      }
-      if (a >= maxlen || units == 0) return false;
-      const int u = q, i = a;
-      if (++q == units) {
-        q = 0;
-        ++a;
-      }
-      const int cb = unit_begin(u), ce = unit_end(u);
-      if (cb + i < ce) {
-        grp = u;
-        tile = R * ng + u / s;
-        c = cb + i;
-        last = c == ce - 1;
-        return true;
-      }
-    }
-  }
+struct EngGeom {
+  int RB;           // bytes per weight row (K / 4)
+  int rs;           // 16-row tiles per stage (full-row mode), 1 in chunked mode
+  int CB;           // bytes of each row per stage (== RB in full-row mode, a multiple of 64 otherwise)
+  int full_rows;    // 1: full-row mode
+  int n_chunks;     // chunks per row
+  int ac_chunks;    // chunks per activation chunk
+  int n_ac;         // activation chunks
+  int x_pitch;      // shared-memory bytes per token of a staged activation chunk
+  int slot_bytes;   // shared-memory bytes a stage occupies (with 64 bytes of slack for a
+                    // 32-byte half step read past the last row)
 };
 
-// The stages of group `grp` in sequence order, with their index `pos` in the producer's
-// sequence: in the full rounds every ng-th stage (tile r * ng + grp, chunks 0 .. nch-1); in
-// the last round unit grp, whose stage i sits at i * units + grp while every unit still has
-// a chunk i (i < lmin), else after the units of the last round that do.
-struct EngOwnStages {
-  int ng, nch, grp, R, s, units, own_full, own_rem, ucb, lmin, rank;
-  int j, rr, cc;
-  ENG_HD EngOwnStages(const EngSched& sc, int grp_)
-      : ng(sc.ng), nch(sc.nch), grp(grp_), R(sc.R), s(sc.s), units(sc.units), own_full(sc.R * sc.nch),
-        own_rem(0), ucb(0), lmin(0), rank(0), j(0), rr(0), cc(0) {
-    if (grp < units) {
-      ucb = sc.unit_begin(grp);
-      own_rem = sc.unit_end(grp) - ucb;
-      lmin = nch / s;
-      for (int u = 0; u < grp; ++u)
-        if (sc.unit_end(u) - sc.unit_begin(u) > lmin) ++rank;
-    }
-  }
-  ENG_HD bool next(int& pos, int& tile, int& c, bool& last) {
-    if (j >= own_full + own_rem) return false;
-    if (j < own_full) {
-      c = cc;
-      tile = rr * ng + grp;
-      pos = (rr * nch + cc) * ng + grp;
-      last = cc == nch - 1;
-      if (++cc == nch) {
-        cc = 0;
-        ++rr;
-      }
-    } else {
-      const int i = j - own_full;
-      c = ucb + i;
-      tile = R * ng + grp / s;
-      pos = R * ng * nch + (i < lmin ? i * units + grp : lmin * units + rank);
-      last = i == own_rem - 1;
-    }
-    ++j;
+// Bytes per token of a staged activation chunk of n in-features: whole 256-in-feature
+// steps (zero-padded), plus 64 so that consecutive tokens fall in different banks.
+ENG_HD int eng_x_pitch_for(int n) { return ((n + 255) / 256) * 256 + 64; }
+
+// Plan a phase of K in-features for T tokens: slot_max bytes per ring slot at most,
+// act_max bytes of shared memory for the staged activations (all T tokens).  Returns false
+// if no geometry fits.
+ENG_HD bool eng_plan(int K, int T, int slot_max, int act_max, EngGeom& g) {
+  g.RB = K / 4;
+  const int RB = g.RB;
+  if (16 * RB + 64 <= slot_max && T * eng_x_pitch_for(K) <= act_max) {
+    g.full_rows = 1;
+    g.CB = RB;
+    int rs = ENG_STAGE_TARGET / (16 * RB);
+    if (rs < 1) rs = 1;
+    if (rs > ENG_MAX_RS) rs = ENG_MAX_RS;
+    while (rs > 1 && 16 * rs * RB + 64 > slot_max) --rs;
+    g.rs = rs;
+    g.n_chunks = 1;
+    g.ac_chunks = 1;
+    g.n_ac = 1;
+    g.x_pitch = eng_x_pitch_for(K);
+    g.slot_bytes = 16 * rs * RB + 64;
     return true;
   }
-};
+  g.full_rows = 0;
+  g.rs = 1;
+  // Largest chunk (multiple of 64 bytes, at most one TMA box row) whose stage and whose
+  // activations (one chunk per activation chunk at least) fit; then even chunks.
+  int cmax = ENG_BOX_MAX_BYTES;
+  while (cmax >= 64 && (16 * cmax + 64 > slot_max || T * eng_x_pitch_for(4 * cmax) > act_max)) cmax -= 64;
+  if (cmax < 64) return false;
+  const int n = (RB + cmax - 1) / cmax;
+  int cb = (RB + n - 1) / n;
+  cb = (cb + 63) / 64 * 64;
+  if (cb > cmax) cb = cmax;
+  g.CB = cb;
+  g.n_chunks = (RB + cb - 1) / cb;
+  int ac = 1;
+  while (ac < g.n_chunks && T * eng_x_pitch_for(4 * cb * (ac + 1)) <= act_max) ++ac;
+  g.ac_chunks = ac;
+  g.n_ac = (g.n_chunks + ac - 1) / ac;
+  g.x_pitch = eng_x_pitch_for(4 * cb * ac);
+  g.slot_bytes = 16 * cb + 64;
+  return true;
+}
+
+// Number of stages of a phase on a CTA with nt tiles.
+ENG_HD int eng_stage_count(const EngGeom& g, int nt, int NT) {
+  const int groups = (nt + g.rs - 1) / g.rs;
+  return groups * NT * g.n_chunks;
+}
 
 }  // namespace bitnet

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   constexpr int NT = FFN ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   volatile __shared__ int s_abort;
+  __shared__ int s_issued;  // stages the producer issued (for the drain after an abort)
   __shared__ uint32_t s_tmem;
   __shared__ float s_f[NT][256];
   __shared__ int s_sq[256];
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   auto empty = [&](int s) { return bars + 8u * (2 * TC_MAX_STAGES + s); };
   auto tm_full = [&](int b) { return bars + 8u * (3 * TC_MAX_STAGES + b); };
   auto tm_empty = [&](int b) { return bars + 8u * (3 * TC_MAX_STAGES + 2 + b); };
+  const uint32_t mma_done = bars + 8u * (3 * TC_MAX_STAGES + 4);  // final commit after an abort
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -153,7 +155,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
       mbar_init(tm_full(b), 1);
       mbar_init(tm_empty(b), 128);
     }
+    mbar_init(mma_done, 1);
     s_abort = 0;
+    s_issued = 0;
     fence_mbar_init();
   }
   if (warp == TC_MMA_WARP) {
@@ -194,6 +198,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
           tma_load_2d(sB(s), &maps.act, kb * TC_BK, tok0, full_tma(s));
 #pragma unroll
           for (int u = 0; u < NT; ++u) tma_load_2d(sP(s, u), &maps.w[FFN ? u : ti], kb * 32, m0, full_tma(s));
+          s_issued = it + 1;
         }
       }
     }
@@ -213,10 +218,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
         }
 #pragma unroll
         for (int u = 0; u < NT; ++u) {
-          uint4 w0, w1;
+          // Rows are 32 bytes apart: lanes 4..7 of each quarter-warp read their row's second
+          // half first, so the eight 16-byte reads of a quarter-warp cover all banks once.
+          const uint32_t sw = (uint32_t)((e >> 2) & 1) * 16u;
           const uint32_t pa = sP(s, u) + r * 32;
-          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w0.x), "=r"(w0.y), "=r"(w0.z), "=r"(w0.w) : "r"(pa));
-          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w1.x), "=r"(w1.y), "=r"(w1.z), "=r"(w1.w) : "r"(pa + 16));
+          const uint4 f0 = lds128(pa + sw), f1 = lds128(pa + (16u - sw));
+          const uint4 w0 = sw ? f1 : f0, w1 = sw ? f0 : f1;
           const uint32_t rowa = sA(s, u) + r * 128;
 #pragma unroll
           for (int gg = 0; gg < 2; ++gg) {
@@ -344,6 +351,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   }
 
   tc_fence_before();
+  __syncthreads();
+  if (s_abort) {
+    // After an abort: let every issued MMA finish (a final commit covers all of them) and
+    // every issued TMA copy land in this CTA's shared memory before TMEM is released and
+    // the CTA exits (fixed drain limit).
+    if (warp == TC_MMA_WARP && lane == 0) {
+      umma_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+    if (warp == TC_TMA_WARP && lane == 0) {
+      const int issued = s_issued;
+      for (int k = (issued > S ? issued - S : 0); k < issued; ++k) mbar_drain(full_tma(k % S), (uint32_t)((k / S) & 1));
+    }
+  }
   __syncthreads();
   if (warp == TC_MMA_WARP) {
     tc_fence_after();

@@ -1,75 +1,89 @@
-// Host check of the decode engine's stage schedule (engine_sched.h), built and run by
-// tests/test_engine_schedule.py.  For every CTA tile count and chunk count in a grid it
-// checks that the producer's sequence holds every (tile, chunk) exactly once, that each
-// group's share of a tile is a contiguous ascending chunk range closed by one `last`
-// flag, and that every group's closed-form stage list (EngOwnStages) is exactly its
-// stages of the producer's sequence, with their sequence positions.
+// Host check of the decode engine's stage geometry (engine_sched.h), built and run by
+// tests/test_engine_schedule.py.  For every row length K (multiples of 128 up to 49152) and
+// token count T (1..16) it checks that the planned stage fits its ring slot, that a chunk is
+// whole 64-byte steps and one TMA box row, that the staged activations fit, and -- walking
+// the stage order the producer and the consumers share for 0..40 tiles and one or two
+// tensors -- that every (tile, tensor, chunk) is streamed exactly once, that every partial
+// sum is flushed exactly once per activation chunk, and that no weight or activation read
+// leaves its buffer.
 #include <cstdio>
 #include <vector>
 
 #include "engine_sched.h"
 
-struct Stage {
-  int grp, tile, c;
-  bool last;
-};
+using namespace bitnet;
 
 int main() {
   int bad = 0, cases = 0;
-  for (int nt = 0; nt <= 48; ++nt) {
-    for (int nch = 1; nch <= 16; ++nch) {
+  auto fail = [&](int K, int T, const char* what) {
+    if (bad < 20) std::printf("FAIL K=%d T=%d: %s\n", K, T, what);
+    ++bad;
+  };
+  for (int K = 128; K <= 49152; K += 128) {
+    for (int T = 1; T <= 16; ++T) {
       ++cases;
-      bitnet::EngSched sc(nt, nch);
-      std::vector<Stage> seq;
-      int grp, tile, c;
-      bool last;
-      while (sc.next(grp, tile, c, last)) seq.push_back({grp, tile, c, last});
-      auto fail = [&](const char* what) {
-        if (bad < 20) std::printf("FAIL nt=%d nch=%d: %s\n", nt, nch, what);
-        ++bad;
-      };
-      if ((int)seq.size() != nt * nch) fail("sequence length");
-      if ((int)seq.size() != bitnet::EngSched(nt, nch).total()) fail("total()");
-      std::vector<int> seen(nt * nch, 0);
-      for (const Stage& st : seq) {
-        if (st.tile < 0 || st.tile >= nt || st.c < 0 || st.c >= nch) {
-          fail("stage out of range");
-          continue;
-        }
-        if (st.grp < 0 || st.grp >= sc.ng) fail("group out of range");
-        ++seen[st.tile * nch + st.c];
+      EngGeom g;
+      if (!eng_plan(K, T, ENG_SLOT_MAX, ENG_ACT_MAX, g)) {
+        fail(K, T, "no geometry");
+        continue;
       }
-      for (int v : seen)
-        if (v != 1) fail("(tile, chunk) not exactly once");
-      for (int g = 0; g < sc.ng; ++g) {
-        // the group's stages in the producer's order, with positions
-        std::vector<int> pos;
-        for (int i = 0; i < (int)seq.size(); ++i)
-          if (seq[i].grp == g) pos.push_back(i);
-        // contiguous ascending chunks per tile, `last` at the end of each run
-        for (size_t k = 0; k < pos.size(); ++k) {
-          const Stage& st = seq[pos[k]];
-          const bool run_ends = k + 1 == pos.size() || seq[pos[k + 1]].tile != st.tile;
-          if (st.last != run_ends) fail("last flag");
-          if (!run_ends && seq[pos[k + 1]].c != st.c + 1) fail("chunks of a run not consecutive");
-        }
-        bitnet::EngOwnStages own(sc, g);
-        int p, t2, c2;
-        bool l2;
-        size_t k = 0;
-        while (own.next(p, t2, c2, l2)) {
-          if (k >= pos.size()) {
-            fail("own stages: too many");
-            break;
+      const int RB = K / 4;
+      if (g.RB != RB) fail(K, T, "RB");
+      if (g.slot_bytes > ENG_SLOT_MAX) fail(K, T, "slot too large");
+      if (T * g.x_pitch > ENG_ACT_MAX) fail(K, T, "activations do not fit");
+      if (g.full_rows) {
+        if (g.CB != RB || g.n_chunks != 1 || g.n_ac != 1 || g.rs < 1 || g.rs > ENG_MAX_RS) fail(K, T, "full-row fields");
+        if (16 * g.rs * RB + 64 > g.slot_bytes) fail(K, T, "full-row slot");
+      } else {
+        if (g.rs != 1 || g.CB % 64 || g.CB > ENG_BOX_MAX_BYTES || g.CB < 64) fail(K, T, "chunk size");
+        if ((long)g.n_chunks * g.CB < RB || (long)(g.n_chunks - 1) * g.CB >= RB) fail(K, T, "chunk count");
+        if (16 * g.CB + 64 > g.slot_bytes) fail(K, T, "chunked slot");
+        if (g.ac_chunks < 1 || (long)g.n_ac * g.ac_chunks < g.n_chunks || (long)(g.n_ac - 1) * g.ac_chunks >= g.n_chunks)
+          fail(K, T, "activation chunks");
+      }
+      // walk the stage order
+      for (int NT = 1; NT <= 2; ++NT) {
+        for (int nt = 0; nt <= 40; ++nt) {
+          std::vector<int> seen(nt * NT * g.n_chunks, 0), flushes(nt * NT * g.n_ac, 0);
+          int stages = 0;
+          for (int ac = 0; ac < g.n_ac; ++ac) {
+            const int wc0 = ac * g.ac_chunks, wc1 = (wc0 + g.ac_chunks < g.n_chunks) ? wc0 + g.ac_chunks : g.n_chunks;
+            const int k0 = 4 * wc0 * g.CB, k1 = (4 * wc1 * g.CB < K) ? 4 * wc1 * g.CB : K;
+            const int staged = (k1 - k0 + 255) / 256 * 256;  // activation bytes per token staged (zero-padded)
+            if (staged + 64 > g.x_pitch) fail(K, T, "staged chunk exceeds the pitch");
+            for (int tg0 = 0; tg0 < nt; tg0 += g.rs) {
+              const int ntg = (g.rs < nt - tg0) ? g.rs : nt - tg0;
+              for (int u = 0; u < NT; ++u) {
+                for (int wc = wc0; wc < wc1; ++wc) {
+                  ++stages;
+                  const int cbytes = (g.CB < RB - wc * g.CB) ? g.CB : RB - wc * g.CB;
+                  const int S = (cbytes + 63) / 64;
+                  const int xoff = 256 * (wc - wc0) * (g.CB / 64);
+                  if (xoff + 256 * S > staged) fail(K, T, "activation read past the staged chunk");
+                  for (int tl = 0; tl < ntg; ++tl) {
+                    // last byte read: row 15 of tile tl, step S-1, lane r = 3
+                    const long last = (long)(tl * 16 + 15) * g.CB + 64L * (S - 1) + 48 + 16;
+                    if (last > g.slot_bytes) fail(K, T, "weight read past the slot");
+                    seen[((tg0 + tl) * NT + u) * g.n_chunks + wc]++;
+                    if (wc == wc1 - 1) flushes[((tg0 + tl) * NT + u) * g.n_ac + ac]++;
+                  }
+                }
+              }
+            }
           }
-          const Stage& st = seq[pos[k]];
-          if (p != pos[k] || t2 != st.tile || c2 != st.c || l2 != st.last) fail("own stage differs");
-          ++k;
+          if (stages != eng_stage_count(g, nt, NT)) fail(K, T, "stage count");
+          for (int v : seen)
+            if (v != 1) fail(K, T, "a (tile, tensor, chunk) not streamed exactly once");
+          for (int v : flushes)
+            if (v != 1) fail(K, T, "a partial sum not flushed exactly once");
         }
-        if (k != pos.size()) fail("own stages: too few");
       }
     }
   }
-  std::printf("%s: %d cases, %d failures\n", bad ? "FAIL" : "OK", cases, bad);
-  return bad != 0;
+  if (bad) {
+    std::printf("%d failures in %d cases\n", bad, cases);
+    return 1;
+  }
+  std::printf("OK %d cases\n", cases);
+  return 0;
 }

@@ -1,10 +1,10 @@
-"""Host test of the decode engine's ring schedule (csrc/engine_sched.h, plain C++).
+"""Host test of the decode engine's stage geometry (csrc/engine_sched.h, plain C++).
 
-The producer warp and the consumer groups of the decode engine must agree exactly on
-which tile and K-chunk every ring stage holds: a disagreement would pair a consumer with
-the wrong weights or leave a barrier waiting.  tests/engine_sched_check.cpp enumerates
-the producer's sequence and each group's closed-form stage list for 49 x 16 shapes and
-checks them against each other; this test builds and runs it with the host compiler.
+The producer warp and the consumer warps of the decode engine walk the same stage order;
+a stage that does not fit its slot, a chunk that is not whole steps, or a read past a
+buffer would pair consumers with the wrong bytes.  tests/engine_sched_check.cpp plans
+every row length up to 49152 for 1..16 tokens and walks the stage order for 0..40 tiles;
+this test builds and runs it with the host compiler.
 """
 from __future__ import annotations
 
@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(os.path.dirname(HERE), "ternary_bitlinear_quantized_b200", "csrc")
 
 
-def test_engine_schedule_covers_every_stage_once_and_groups_agree(tmp_path):
+def test_engine_stage_geometry_fits_and_covers_every_stage_once(tmp_path):
     cxx = shutil.which("g++") or shutil.which("c++")
     if cxx is None:
         pytest.skip("no host C++ compiler")

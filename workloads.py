@@ -124,3 +124,26 @@ def block_inputs(shape: BlockShape, T: int, seed: int = 0, outliers: bool = Fals
         d["g_attn_sub_norm"] = gain(shape.n_q, seed, f"{shape.name}/attn_sub_norm", device)
         d["attn_out"] = activations(T, shape.n_q, seed, f"{shape.name}/attn_out", outliers, device)
     return d
+
+
+# Attention at decode: the heads of the block shapes (2B4T: 20 query / 5 key-value heads,
+# 70B: 64 / 8, head size 128) over a KV cache of synthetic earlier tokens.  The pages give no
+# context length; 4096 cached positions stand in for a long prompt.
+ATTN_SHAPES = {"2b4t": (20, 5), "70b": (64, 8)}
+ATTN_CONTEXT = 4096
+
+
+def attention_inputs(T: int, Hq: int, Hkv: int, L_max: int, pos0: int, seed: int = 0, device: str = "cpu") -> dict:
+    """New tokens' q [T, Hq, 128], k and v [T, Hkv, 128] (bf16 ~ N(0, 1), the projections'
+    outputs) and bf16 caches [Hkv, L_max, 128] whose first pos0 rows hold earlier tokens'
+    (already rotated) keys and values ~ N(0, 1); the other rows are zero."""
+    d = {}
+    for nm, h in (("q", Hq), ("k", Hkv), ("v", Hkv)):
+        g = _gen(seed, f"attn/{nm}", device)
+        d[nm] = torch.randn(T, h, 128, generator=g, device=device).to(torch.bfloat16)
+    for nm in ("k_cache", "v_cache"):
+        g = _gen(seed, f"attn/{nm}", device)
+        c = torch.zeros(Hkv, L_max, 128, dtype=torch.bfloat16, device=device)
+        c[:, :pos0] = torch.randn(Hkv, pos0, 128, generator=g, device=device).to(torch.bfloat16)
+        d[nm] = c
+    return d
