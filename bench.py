@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--prefill-workload", default="ffn_32b_t4096", choices=sorted(workloads.WORKLOADS) + ["none"],
                     help="prefill workload reported in the line's `prefill` object ('none' to skip)")
     ap.add_argument("--prefill-steps", type=int, default=30)
+    ap.add_argument("--attention", default="70b", choices=["none"] + sorted(workloads.ATTN_SHAPES),
+                    help="heads of the block whose decode attention is reported in the `attention` object")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle sample")
     ap.add_argument("--seed", type=int, default=0)
@@ -556,6 +558,62 @@ def measure(name: str, args, world: int, use_graph: bool, steps: int, int8_peak=
     return fields, clocks
 
 
+def measure_attention(shape: str, steps: int, warmup: int):
+    """Decode attention of one block (T = 1): rotary embedding + cache append of the new token,
+    then causal GQA attention over ATTN_CONTEXT cached positions.  Bound by the cache read:
+    2 x Hkv x L x 256 bytes per step (keys and values, bf16)."""
+    import ternary_bitlinear_quantized_b200 as tb
+    Hq, Hkv = workloads.ATTN_SHAPES[shape]
+    L = workloads.ATTN_CONTEXT
+    T, pos0 = 1, L - 1
+    dev = f"cuda:{torch.cuda.current_device()}"
+    # several caches rotate so that the reads come from HBM (each 2 x Hkv x L x 256 bytes)
+    cache_bytes = 2 * Hkv * L * 256
+    R = max(2, math.ceil(2 * L2_BYTES / cache_bytes) + 1)
+    d = workloads.attention_inputs(T, Hq, Hkv, L, pos0, seed=0, device=dev)
+    caches = [(d["k_cache"].clone(), d["v_cache"].clone()) for _ in range(R)]
+    q_rot = torch.empty(T, Hq, 128, dtype=torch.float32, device=dev)
+    out = torch.empty(T, Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(tb.attention_workspace_bytes(T, Hq, Hkv, L), dtype=torch.uint8, device=dev)
+
+    def one(c):
+        kc, vc = caches[c]
+        tb.rope_kv_append(d["q"], d["k"], d["v"], pos0, 10000.0, kc, vc, q_rot=q_rot)
+        tb.attention_decode(q_rot, kc, vc, pos0, out=out, ws=ws)
+
+    for c in range(R):
+        one(c)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for c in range(R):
+            one(c)
+    torch.cuda.synchronize()
+    reps = max(1, steps // R)
+    for _ in range(max(1, warmup // R)):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * R)
+    (ms,) = max_over_ranks([ms])
+    hbm, _, src = peaks()
+    gbs = cache_bytes / (ms / 1e3) / 1e9
+    return {"workload": f"attention_{shape}_decode_t1_ctx{L}", "metric": "KV-cache HBM GB/s (decode attention)",
+            "value": gbs, "unit": "GB/s", "us_per_step": ms * 1e3, "steps": reps * R,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "bytes_per_step": cache_bytes, "peak_source": f"{src} hbm_gbs",
+                         "kernels": "k_rope_append + k_attn_partial + k_attn_combine"},
+            "l2": f"caches rotated over {R} copies ({R * cache_bytes / 1e6:.0f} MB > 2x L2)",
+            "gpu_launches": 3 * reps * R}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -601,6 +659,8 @@ def main():
                    ("metric", "value", "unit", "steps", "ms_per_step", "config", "roofline", "e2e", "gpu_launches")},
                    "clocks": pclocks, "int8_peak_measured_tops": int8_peak}
 
+    attention = measure_attention(args.attention, 200, 20) if args.attention != "none" else None
+
     cpu = None
     if rank == 0 and world == 1:
         cpu = oracle_sample(args.workload, args.seed, args.cpu_seconds, single_thread_seconds=args.cpu_seconds / 2)
@@ -622,6 +682,8 @@ def main():
         }
         if prefill is not None:
             line["prefill"] = prefill
+        if attention is not None:
+            line["attention"] = attention
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

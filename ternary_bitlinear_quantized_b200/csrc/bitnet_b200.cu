@@ -365,6 +365,14 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   }
   qs = (qs + 127) / 128 * 128;
   acc_ints = (acc_ints + 3) / 4 * 4;
+  int sub_rows = 0;  // rows of h a CTA keeps for a SUBNORM phase, and their gain
+  for (int i = 0; i < a.n_phases; ++i)
+    if (a.ph[i].kind == PH_GEMV_FFN && a.ph[i].pmax != nullptr) {
+      const int r = (a.ph[i].n_tiles + grid - 1) / grid * GEMV_ROWS;
+      if (r > sub_rows) sub_rows = r;
+    }
+  xs = (xs + 3) / 4 * 4;  // keep what follows 16-byte aligned
+  const int sub_floats = (a.T + 1) * sub_rows;
   const int tg = a.T <= 8 ? 1 : 2;
   void (*kern)(const EngArgs, const EngMaps) = tg == 1 ? k_engine<1> : k_engine<2>;
   cudaFuncAttributes fa;
@@ -375,7 +383,7 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int budget = max_optin - (int)fa.sharedSizeBytes - 1024;  // 1024: ring alignment
-  const int ring = budget - acc_ints * 4 - qs - xs * 4;
+  const int ring = budget - acc_ints * 4 - qs - xs * 4 - sub_floats * 4;
   if (slot == 0) slot = 1024;  // no product phase (not planned by this library, but harmless)
   int slots = ring / (slot + 16);
   if (slots * slot > ENG_RING_MAX) slots = ENG_RING_MAX / slot;
@@ -386,7 +394,9 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   a.acc_ints = acc_ints;
   a.qs_bytes = qs;
   a.xs_floats = xs;
-  const size_t smem = 1024 + (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4;
+  a.sub_rows = sub_rows;
+  const size_t smem =
+      1024 + (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4 + (size_t)sub_floats * 4;
   e = opt_in_smem((const void*)kern, 6 + tg - 1);
   if (e != cudaSuccess) return cuda_fail(e, "k_engine attribute");
   // Grid barriers need every CTA resident at once: one CTA per SM must fit.
@@ -765,9 +775,13 @@ bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size
   return BITNET_OK;
 }
 
-// Per-CTA partial reductions of the distributed sub-norm after the counters: max [T][G]
-// fp32 and fixed-point sums [T][G] int64, G = ENG_MAX_GRID.
-static size_t ffn_partials_bytes(int64_t T) { return align_up((size_t)T * ENG_MAX_GRID * 4) + (size_t)T * ENG_MAX_GRID * 8; }
+// Per-CTA partial reductions of the distributed sub-norm after the counters (G = ENG_MAX_GRID):
+// max |h| [T][G] fp32, max |y| [T][G] fp32, candidate fixed-point sums [T][G][ENG_SUB_CAND]
+// int64, fallback sums [T][G] int64.
+static size_t ffn_partials_bytes(int64_t T) {
+  return 2 * align_up((size_t)T * ENG_MAX_GRID * 4) + align_up((size_t)T * ENG_MAX_GRID * ENG_SUB_CAND * 8) +
+         (size_t)T * ENG_MAX_GRID * 8;
+}
 
 size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I) {
   size_t off[FFN_WS_SLOTS];
@@ -803,19 +817,25 @@ static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32,
     eng_src_global(gate_up, q_x, s_x, sum_x);
     gate_up.wait_barrier = qp.arrive_barrier;
   }
-  gate_up.arrive_barrier = bar++;
   const int64_t nH[1] = {H};
   void* o[1] = {out};
   EngPhase down = eng_gemv((int)I, false, 1, &p_down, nH, o, nullptr, ot, act, nullptr);
   if (eng_local_ok(T, I)) {
+    gate_up.arrive_barrier = bar++;
     ea.ph[ea.n_phases++] = gate_up;
     eng_src_local(down, h, 1, g_sub, q_h, s_h, sum_h);
     down.wait_barrier = gate_up.arrive_barrier;
   } else {
-    // ffn_sub_norm spread over the grid: every CTA reduces the rows of h it produced.
-    float* pmax = reinterpret_cast<float*>(ws + off[7] + ENG_COUNTER_BYTES);
-    long long* psum = reinterpret_cast<long long*>(ws + off[7] + ENG_COUNTER_BYTES + align_up((size_t)T * ENG_MAX_GRID * 4));
+    // ffn_sub_norm spread over the grid: every CTA reduces the rows of h it produced (kept
+    // in its shared memory, so the SUBNORM phase starts without waiting for the others).
+    uint8_t* pb = ws + off[7] + ENG_COUNTER_BYTES;
+    float* pmax = reinterpret_cast<float*>(pb);
+    float* pmax2 = reinterpret_cast<float*>(pb + align_up((size_t)T * ENG_MAX_GRID * 4));
+    long long* psum = reinterpret_cast<long long*>(pb + 2 * align_up((size_t)T * ENG_MAX_GRID * 4));
+    long long* psum_fb = reinterpret_cast<long long*>(pb + 2 * align_up((size_t)T * ENG_MAX_GRID * 4) +
+                                                      align_up((size_t)T * ENG_MAX_GRID * ENG_SUB_CAND * 8));
     gate_up.pmax = pmax;
+    gate_up.sub_gain = g_sub;
     ea.ph[ea.n_phases++] = gate_up;
     EngPhase sp;
     memset(&sp, 0, sizeof(sp));
@@ -829,10 +849,13 @@ static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32,
     sp.s = s_h;
     sp.sq = sum_h;
     sp.pmax = pmax;
+    sp.pmax2 = pmax2;
     sp.psum = psum;
-    sp.wait_barrier = gate_up.arrive_barrier;
+    sp.psum_fb = psum_fb;
+    sp.wait_barrier = -1;
     sp.bar_a = bar++;
     sp.bar_b = bar++;
+    sp.bar_fb = bar++;
     sp.arrive_barrier = bar++;
     ea.ph[ea.n_phases++] = sp;
     eng_src_global(down, q_h, s_h, sum_h);

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "../../include/bitnet_b200.h"
+#include "fixed_point.h"
 
 #define BN_DEV __device__ __forceinline__
 #define BN_HOST_DEV __host__ __device__
@@ -131,6 +132,14 @@ BN_DEV void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t ba
                : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (both 16-byte aligned), completed by
+// cp_async_wait_all in the issuing thread.
+BN_DEV void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+BN_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+BN_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Named barrier over `count` threads (a multiple of 32).
 BN_DEV void named_sync(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 // Named barrier that also returns whether `pred` was true in any of the threads.
@@ -169,6 +178,8 @@ BN_DEV float fixed_point_mean(long long S, int e, long long n) {
 }
 
 BN_DEV float bf16_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+
+// The integer terms of the exact fixed-point sums: fixed_point.h.
 
 // ---------------------------------------------------------------- reductions
 BN_DEV float warp_max(float v) {

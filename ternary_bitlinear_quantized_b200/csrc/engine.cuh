@@ -78,12 +78,17 @@ struct EngPhase {
   int out_dtype, act;
   float* h;           // FFN output [T, N] fp32
   int wait_barrier, arrive_barrier;  // -1: none
-  // SUBNORM (and the GEMV_FFN phase before it): per-CTA partials [T][gridDim.x] of
-  // max |h| then max |y| (pmax) and of the fixed-point sum of h^2 (psum); the SUBNORM
-  // phase's two inner grid barriers.
+  // SUBNORM (and the GEMV_FFN phase before it): per-CTA partials of max |h| (pmax [T][G]),
+  // of the fixed-point sum of h^2 on ENG_SUB_CAND candidate grids (psum [T][G][ENG_SUB_CAND]),
+  // of the sum on the global grid when the candidates do not cover it (psum_fb [T][G]) and of
+  // max |y| (pmax2 [T][G]); the SUBNORM phase's inner grid barriers; the sub-norm gain, which
+  // the gate/up phase prefetches for its rows (sub_gain).
   float* pmax;
   long long* psum;
-  int bar_a, bar_b;
+  long long* psum_fb;
+  float* pmax2;
+  const float* sub_gain;
+  int bar_a, bar_b, bar_fb;
   EngGeom g;  // stage geometry of a product phase (engine_sched.h)
 };
 
@@ -99,6 +104,8 @@ struct alignas(16) EngArgs {
   int n_phases;
   unsigned* counters;  // ENG_MAX_BARRIERS + 1 words in the workspace (last: exit count)
   int n_slots, slot_bytes, acc_ints, qs_bytes, xs_floats;
+  int sub_rows;  // rows of h a CTA keeps for the SUBNORM phase (0: none)
+  int pad_[3];
   EngPhase ph[ENG_MAX_PHASES];
 };
 
@@ -225,16 +232,12 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
     float ms = 0.0f;
     if (am > 0.0f) {
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
-      const double p2e = pow2_f64(e);
       long long part = 0;
 #pragma unroll
       for (int j = 0; j < ENG_REG_GROUPS; ++j) {
         if (8 * (tid + ENG_CONS * j) < K) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const double d = (double)v[j][i];
-            part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
-          }
+          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], e);
         }
       }
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
@@ -312,12 +315,8 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
     float ms = 0.0f;
     if (am > 0.0f) {
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
-      const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int kk = tid; kk < K; kk += ENG_CONS) {
-        const double d = (double)xs[kk];
-        part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
-      }
+      for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term(xs[kk], e);
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
@@ -390,10 +389,13 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 
 // ------------------------------------------------------------------ distributed sub-norm
 // Per-token scratch of the SUBNORM phase in shared memory.
+constexpr int ENG_SUB_CAND = 8;  // candidate grids per CTA: local exponent e_c, e_c - 1, .., e_c - 7
 struct SubScratch {
-  unsigned mx[ENG_MAX_T];  // max |h|, then max |y| (non-negative floats as bits)
-  unsigned my[ENG_MAX_T];
+  unsigned mx[ENG_MAX_T];  // the global max |h| (non-negative floats as bits)
+  unsigned my[ENG_MAX_T];  // max |y|
   unsigned long long sum[ENG_MAX_T];
+  int e[ENG_MAX_T];        // the row's grid exponent
+  int fallback;
   float inv[ENG_MAX_T];
   float scale[ENG_MAX_T];
   int sq[ENG_MAX_T];
@@ -407,84 +409,123 @@ BN_DEV bool grid_step(unsigned* ctr) {
   return !named_sync_or(1, ENG_CONS, !ok);
 }
 
-// ffn_sub_norm + absmax int8 of h [T, K] (fp32, plain order) into p.q / p.s / p.sq, every
-// row split over the grid: this CTA owns the 16-row tiles [tb, te) it produced in the
-// gate/up phase, whose epilogue left max |h| of those rows in p.pmax[t][cta].  The same
-// arithmetic as quant_row, with each reduction finished across the grid: max |h| ->
-// exponent e -> exact fixed-point sum of h^2 -> inv -> y = h * inv * g -> max |y| -> s_x
-// -> q.  Maxima and integer sums are order-free, so the result does not depend on the
-// split.  p.sq must be zero on entry (the kernel clears it before the gate/up phase).
+// ffn_sub_norm + absmax int8 of h [T, K] (fp32) into p.q / p.s / p.sq, every row split over
+// the grid: this CTA owns the rows of the 16-row tiles [tb, te) it produced in the gate/up
+// phase, whose epilogue kept them in shared memory (hs [T][sub_rows]) and which prefetched the
+// matching gain slice (gs).  The same arithmetic as quant_row, with each reduction finished
+// across the grid:
+//   1. the CTA's max |h| M_c and its fixed-point sums of h^2 on the grids of the exponents
+//      e_c, e_c - 1, .., e_c - 7 (e_c from M_c and the row length) -> published; grid barrier;
+//   2. the global max M gives the row's grid e <= e_c; when every CTA's candidates include
+//      e (or M_c = 0, whose sum is 0 on any grid) the sum is the sum of those candidates,
+//      else (uniformly, from the same published maxima) every CTA sums on e itself and a
+//      second barrier publishes those sums;
+//   3. inv, max |y| of the CTA's rows -> published; grid barrier; 4. s_x and q of its rows.
+// Maxima and integer sums are order-free, so the result does not depend on the split.
+// p.sq must be zero on entry (the kernel clears it before the gate/up phase).
 __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, int tb, int te, unsigned* counters,
-                                         SubScratch& S) {
-  const int G = gridDim.x, K = p.K, tid = threadIdx.x, nt = te - tb;
-  const float* h = reinterpret_cast<const float*>(p.x);
+                                         SubScratch& S, const float* hs, const float* gs, int sub_rows) {
+  const int G = gridDim.x, K = p.K, tid = threadIdx.x, nrows = (te - tb) * GEMV_ROWS;
+  const int warp = tid >> 5, lane = tid & 31;
+  cp_async_wait_all();  // this thread's part of the gain slice
   if (tid < T) {
-    S.mx[tid] = S.my[tid] = 0u;
+    S.my[tid] = 0u;
     S.sum[tid] = 0ull;
-    S.sq[tid] = 0;
+  }
+  if (tid == 0) S.fallback = 0;
+  // 1. this CTA's max |h| and its candidate sums, a warp per token
+  for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+    const float* hr = hs + t * sub_rows;
+    float m = 0.0f;
+    for (int r = lane; r < nrows; r += 32) m = fmaxf(m, fabsf(hr[r]));
+    m = warp_max(m);
+    long long c[ENG_SUB_CAND];
+#pragma unroll
+    for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] = 0;
+    if (m > 0.0f && p.gain != nullptr) {
+      const int e = fixed_point_exponent(__dmul_rn((double)m, (double)m), K);
+      for (int r = lane; r < nrows; r += 32) {
+        const float v = hr[r];
+#pragma unroll
+        for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] += fixed_sq_term(v, e - d);
+      }
+    }
+#pragma unroll
+    for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] = warp_sum_ll(c[d]);
+    if (lane == 0) {
+      p.pmax[t * G + blockIdx.x] = m;
+      if (p.gain != nullptr)
+#pragma unroll
+        for (int d = 0; d < ENG_SUB_CAND; ++d) p.psum[((long long)t * G + blockIdx.x) * ENG_SUB_CAND + d] = c[d];
+    }
+  }
+  if (!grid_step(counters + p.bar_a)) return false;
+  // 2. the global max; the sum from the candidates when they cover the global grid
+  constexpr int PER = (ENG_MAX_T * ENG_MAX_GRID + ENG_CONS - 1) / ENG_CONS;
+  float pm[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int i = tid + j * ENG_CONS;
+    pm[j] = i < T * G ? __ldcg(p.pmax + i) : 0.0f;
+  }
+  if (tid < T) S.mx[tid] = 0u;
+  cons_sync();
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int i = tid + j * ENG_CONS;
+    if (i < T * G) atomicMax(&S.mx[i / G], __float_as_uint(pm[j]));
   }
   cons_sync();
-  for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.mx[i / G], __float_as_uint(__ldcg(p.pmax + i)));
+  if (tid < T) {
+    const float am = __uint_as_float(S.mx[tid]);
+    S.e[tid] = am > 0.0f ? fixed_point_exponent(__dmul_rn((double)am, (double)am), K) : 0;
+  }
   cons_sync();
   if (p.gain != nullptr) {
-    // exact fixed-point sum of h^2 over this CTA's rows
-    for (int i = tid; i < T * nt; i += ENG_CONS) {
-      const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
-      const float am = __uint_as_float(S.mx[t]);
-      if (am > 0.0f) {
-        const double p2e = pow2_f64(fixed_point_exponent(__dmul_rn((double)am, (double)am), K));
-        long long part = 0;
 #pragma unroll
-        for (int j = 0; j < GEMV_ROWS; j += 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const double d = (double)vv[k];
-            part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
-          }
-        }
-        atomicAdd(&S.sum[t], (unsigned long long)part);
+    for (int j = 0; j < PER; ++j) {
+      const int i = tid + j * ENG_CONS;
+      if (i < T * G && pm[j] > 0.0f) {
+        const int t = i / G;
+        const int d = fixed_point_exponent(__dmul_rn((double)pm[j], (double)pm[j]), K) - S.e[t];
+        if (d >= ENG_SUB_CAND)
+          S.fallback = 1;
+        else
+          atomicAdd(&S.sum[t], (unsigned long long)__ldcg(p.psum + (long long)i * ENG_SUB_CAND + d));
       }
     }
     cons_sync();
-    if (tid < T) p.psum[tid * G + blockIdx.x] = (long long)S.sum[tid];
-    if (!grid_step(counters + p.bar_a)) return false;
-    if (tid < T) S.sum[tid] = 0ull;
-    cons_sync();
-    for (int i = tid; i < T * G; i += ENG_CONS) atomicAdd(&S.sum[i / G], (unsigned long long)__ldcg(p.psum + i));
-    cons_sync();
+    if (S.fallback) {  // the same decision in every CTA (it follows from the published maxima)
+      for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+        long long c = 0;
+        if (S.mx[t] != 0u)
+          for (int r = lane; r < nrows; r += 32) c += fixed_sq_term(hs[t * sub_rows + r], S.e[t]);
+        c = warp_sum_ll(c);
+        if (lane == 0) p.psum_fb[t * G + blockIdx.x] = c;
+      }
+      if (!grid_step(counters + p.bar_fb)) return false;
+      if (tid < T) S.sum[tid] = 0ull;
+      cons_sync();
+      for (int i = tid; i < T * G; i += ENG_CONS) atomicAdd(&S.sum[i / G], (unsigned long long)__ldcg(p.psum_fb + i));
+      cons_sync();
+    }
+    // 3. inv and max |y| of this CTA's rows
     if (tid < T) {
       const float am = __uint_as_float(S.mx[tid]);
-      float ms = 0.0f;
-      if (am > 0.0f)
-        ms = fixed_point_mean((long long)S.sum[tid], fixed_point_exponent(__dmul_rn((double)am, (double)am), K), K);
+      const float ms = am > 0.0f ? fixed_point_mean((long long)S.sum[tid], S.e[tid], K) : 0.0f;
       S.inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     }
     cons_sync();
-    // max |y| over this CTA's rows
-    for (int i = tid; i < T * nt; i += ENG_CONS) {
-      const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
+    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
       const float inv = S.inv[t];
       float m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < GEMV_ROWS; j += 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
-        const float4 g = __ldg(reinterpret_cast<const float4*>(p.gain + r0 + j));
-        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.x, inv), g.x)));
-        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.y, inv), g.y)));
-        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.z, inv), g.z)));
-        m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(v.w, inv), g.w)));
-      }
-      atomicMax(&S.my[t], __float_as_uint(m));
+      for (int r = lane; r < nrows; r += 32) m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(hs[t * sub_rows + r], inv), gs[r])));
+      m = warp_max(m);
+      if (lane == 0) p.pmax2[t * G + blockIdx.x] = m;
     }
-    cons_sync();
-    // every CTA has read max |h| before passing bar_a, so pmax can hold max |y| now
-    if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
     if (!grid_step(counters + p.bar_b)) return false;
-    if (tid < T) S.my[tid] = 0u;
     cons_sync();
-    for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.my[i / G], __float_as_uint(__ldcg(p.pmax + i)));
+    for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.my[i / G], __float_as_uint(__ldcg(p.pmax2 + i)));
     cons_sync();
   } else {
     if (tid < T) {
@@ -495,38 +536,28 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
   }
   if (tid < T) S.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(S.my[tid]), 1e-5f));
   cons_sync();
-  // q of this CTA's rows, 16 bytes per tile row group
-  for (int i = tid; i < T * nt; i += ENG_CONS) {
-    const int t = i / nt, r0 = (tb + i - t * nt) * GEMV_ROWS;
+  // 4. q of this CTA's rows, four at a time, a warp per token
+  for (int t = warp; t < T; t += ENG_CONS_WARPS) {
     const float inv = S.inv[t], sc = S.scale[t];
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
     int sum = 0;
-#pragma unroll
-    for (int j = 0; j < GEMV_ROWS; j += 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (long long)t * K + r0 + j));
-      float y[4] = {v.x, v.y, v.z, v.w};
-      if (p.gain != nullptr) {
-        const float4 g = __ldg(reinterpret_cast<const float4*>(p.gain + r0 + j));
-        y[0] = __fmul_rn(__fmul_rn(v.x, inv), g.x);
-        y[1] = __fmul_rn(__fmul_rn(v.y, inv), g.y);
-        y[2] = __fmul_rn(__fmul_rn(v.z, inv), g.z);
-        y[3] = __fmul_rn(__fmul_rn(v.w, inv), g.w);
-      }
+    for (int r = 4 * lane; r < nrows; r += 128) {
+      uint32_t w = 0u;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        int qv = __float2int_rn(__fmul_rn(y[k], sc));
+        float y = hs[t * sub_rows + r + k];
+        if (p.gain != nullptr) y = __fmul_rn(__fmul_rn(y, inv), gs[r + k]);
+        int qv = __float2int_rn(__fmul_rn(y, sc));
         qv = min(127, max(-128, qv));
         sum += qv;
-        w[j >> 2] |= (uint32_t)(qv & 0xFF) << (8 * k);
+        w |= (uint32_t)(qv & 0xFF) << (8 * k);
       }
+      *reinterpret_cast<uint32_t*>(p.q + (long long)t * K + tb * GEMV_ROWS + r) = w;
     }
-    *reinterpret_cast<uint4*>(p.q + (long long)t * K + r0) = make_uint4(w[0], w[1], w[2], w[3]);
-    atomicAdd(&S.sq[t], sum);
-  }
-  cons_sync();
-  if (tid < T) {
-    atomicAdd(p.sq + tid, S.sq[tid]);
-    if (blockIdx.x == 0) p.s[tid] = S.scale[tid];
+    sum = warp_sum_i(sum);
+    if (lane == 0) {
+      atomicAdd(p.sq + t, sum);
+      if (blockIdx.x == 0) p.s[t] = sc;
+    }
   }
   return true;
 }
@@ -641,7 +672,6 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   __shared__ int32_t s_loc_sq[ENG_MAX_T];
   __shared__ float s_beta[ENG_MAX_PHASES][4];
   __shared__ SubScratch s_sub;
-  __shared__ unsigned s_hmax[ENG_MAX_T];  // max |h| of this CTA's rows (gate/up epilogue)
   __shared__ int s_issued;                // stages the producer issued (for the drain on exit)
 
   // TMA boxes land 1024-byte aligned.
@@ -650,6 +680,8 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   int* acc = reinterpret_cast<int*>(ring + a.n_slots * a.slot_bytes + 16 * a.n_slots);
   int8_t* qs = reinterpret_cast<int8_t*>(acc + a.acc_ints);  // activations, layout eng_perm
   float* xs = reinterpret_cast<float*>(qs + a.qs_bytes);     // fp32 staging of one activation row
+  float* hs = xs + a.xs_floats;                              // this CTA's rows of h [T][sub_rows]
+  float* gs = hs + a.T * a.sub_rows;                         // and the sub-norm gain of those rows
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (a.n_slots + s); };
 
@@ -664,15 +696,6 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     s_abort = 0;
     s_issued = 0;
     fence_mbar_init();
-  }
-  if (threadIdx.x < ENG_MAX_PHASES * 4) {  // per-tensor scales (weights: no dependency wait needed)
-    const int pi = threadIdx.x >> 2, u = threadIdx.x & 3;
-    float b = 0.0f;
-    if (pi < a.n_phases && ph_is_gemv(a.ph[pi].kind) && u < a.ph[pi].n_tensors) {
-      const EngTensor& t = a.ph[pi].t[u];
-      b = __ldg(reinterpret_cast<const float*>(t.packed + (long long)t.N * (a.ph[pi].K >> 2)));
-    }
-    s_beta[pi][u] = b;
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -765,6 +788,17 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     // ------------------------------------------------------------ consumers
     const int gid = lane >> 2, r = lane & 3;
     const int t_a = gid, t_b = 8 + gid;
+    if (threadIdx.x < ENG_MAX_PHASES * 4) {
+      // per-tensor scales (weights: no dependency wait needed); read by the epilogues, after
+      // the named barriers of the first phase
+      const int pi = threadIdx.x >> 2, u = threadIdx.x & 3;
+      float b = 0.0f;
+      if (pi < a.n_phases && ph_is_gemv(a.ph[pi].kind) && u < a.ph[pi].n_tensors) {
+        const EngTensor& t = a.ph[pi].t[u];
+        b = __ldg(reinterpret_cast<const float*>(t.packed + (long long)t.N * (a.ph[pi].K >> 2)));
+      }
+      s_beta[pi][u] = b;
+    }
     pdl_wait();  // activations and workspace belong to the previous kernel until now
     int slot = 0;       // ring position of the next stage
     uint32_t par = 0;   // and the phase parity of its barriers
@@ -797,7 +831,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
       if (p.kind == PH_SUBNORM) {
         int tb0, te0;
         tile_range(p, tb0, te0);
-        if (!eng_subnorm(p, T, a.eps, tb0, te0, a.counters, s_sub)) {
+        if (!eng_subnorm(p, T, a.eps, tb0, te0, a.counters, s_sub, hs, gs, a.sub_rows)) {
           s_abort = 1;
           break;
         }
@@ -836,7 +870,12 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         }
       }
       for (int i = threadIdx.x; i < nt * NT * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
-      if (threadIdx.x < T) s_hmax[threadIdx.x] = 0u;
+      if (p.pmax != nullptr && p.sub_gain != nullptr) {
+        // the SUBNORM phase's gain for this CTA's rows, fetched while the products run
+        for (int i = threadIdx.x; i < nt * GEMV_ROWS / 4; i += ENG_CONS)
+          cp_async16(smem_addr(gs + 4 * i), p.sub_gain + (long long)tb * GEMV_ROWS + 4 * i);
+        cp_async_commit();
+      }
 
       {
         const uint32_t qs_s = smem_addr(qs);
@@ -918,15 +957,11 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
           const float vU = dequant(accU, __fdiv_rn(betaU, sx));
           const float hv = ffn_act(vA, vU, p.act);
           p.h[(long long)t * N + n] = hv;
-          if (p.pmax != nullptr) atomicMax(&s_hmax[t], __float_as_uint(fabsf(hv)));
+          if (p.pmax != nullptr) hs[t * a.sub_rows + tl2 * GEMV_ROWS + row] = hv;  // kept for the SUBNORM phase
         } else {
           if (p.t[ti].out) store_out(p.t[ti].out, p.out_dtype, (long long)t * N + n, vA);
           if (p.t[ti].acc_debug) p.t[ti].acc_debug[(long long)t * N + n] = accA;
         }
-      }
-      if (p.pmax != nullptr) {  // max |h| of this CTA's rows, for the SUBNORM phase
-        cons_sync();
-        if (threadIdx.x < T) p.pmax[threadIdx.x * gridDim.x + blockIdx.x] = __uint_as_float(s_hmax[threadIdx.x]);
       }
       if (p.arrive_barrier >= 0)
         grid_arrive(a.counters + p.arrive_barrier);
@@ -935,6 +970,7 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     }
   }
 
+  cp_async_wait_all();
   __syncthreads();
   // After an abort, copies the producer issued may still be in flight into this CTA's shared
   // memory: wait for every slot's last fill to land (fixed limit) before the CTA exits.

@@ -55,16 +55,11 @@ __global__ void __launch_bounds__(SHARD_THREADS) k_shard_sumsq(const float* __re
     const float am = amax_g[t];
     long long part = 0;
     if (am > 0.0f) {
-      const double p2e = pow2_f64(fixed_point_exponent(__dmul_rn((double)am, (double)am), K_total));
+      const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K_total);
       const float4* row = reinterpret_cast<const float4*>(h + (long long)t * Ks);
       for (int i = threadIdx.x; i < Ks / 4; i += blockDim.x) {
         const float4 v = row[i];
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const double d = (double)vv[j];
-          part += __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
-        }
+        part += fixed_sq_term(v.x, e) + fixed_sq_term(v.y, e) + fixed_sq_term(v.z, e) + fixed_sq_term(v.w, e);
       }
     }
     part = block_reduce(part, red, AddOpLL());
