@@ -7,7 +7,6 @@
 #include <stdint.h>
 
 #include "../../include/bitnet_b200.h"
-#include "fixed_point.h"
 
 #define BN_DEV __device__ __forceinline__
 #define BN_HOST_DEV __host__ __device__
@@ -179,7 +178,15 @@ BN_DEV float fixed_point_mean(long long S, int e, long long n) {
 
 BN_DEV float bf16_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
 
-// The integer terms of the exact fixed-point sums: fixed_point.h.
+// The terms of the exact fixed-point sums on the grid 2^-e (p2e = 2^e): rint(v^2 2^e) and
+// rint(|v| 2^e) for an fp32 v, in fp64, where v^2 and the scaling are exact; then rounded
+// half to even to an integer.  Valid while the result is below 2^62, which the choice of e
+// guarantees.
+BN_DEV long long fixed_sq_term(float v, double p2e) {
+  const double d = (double)v;
+  return __double2ll_rn(__dmul_rn(__dmul_rn(d, d), p2e));
+}
+BN_DEV long long fixed_abs_term(float v, double p2e) { return __double2ll_rn(__dmul_rn((double)fabsf(v), p2e)); }
 
 // ---------------------------------------------------------------- reductions
 BN_DEV float warp_max(float v) {

@@ -232,12 +232,13 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
     float ms = 0.0f;
     if (am > 0.0f) {
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
+      const double p2e = pow2_f64(e);
       long long part = 0;
 #pragma unroll
       for (int j = 0; j < ENG_REG_GROUPS; ++j) {
         if (8 * (tid + ENG_CONS * j) < K) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], e);
+          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
         }
       }
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
@@ -315,8 +316,9 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
     float ms = 0.0f;
     if (am > 0.0f) {
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
+      const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term(xs[kk], e);
+      for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term(xs[kk], p2e);
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
@@ -391,10 +393,11 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 // Per-token scratch of the SUBNORM phase in shared memory.
 constexpr int ENG_SUB_CAND = 8;  // candidate grids per CTA: local exponent e_c, e_c - 1, .., e_c - 7
 struct SubScratch {
-  unsigned mx[ENG_MAX_T];  // the global max |h| (non-negative floats as bits)
+  unsigned mx[ENG_MAX_T];  // max |h|: this CTA's, then the row's (non-negative floats as bits)
   unsigned my[ENG_MAX_T];  // max |y|
   unsigned long long sum[ENG_MAX_T];
-  int e[ENG_MAX_T];        // the row's grid exponent
+  unsigned long long cand[ENG_MAX_T][ENG_SUB_CAND];  // this CTA's sums on its candidate grids
+  int e[ENG_MAX_T];        // the grid exponent: this CTA's, then the row's
   int fallback;
   float inv[ENG_MAX_T];
   float scale[ENG_MAX_T];
@@ -427,38 +430,50 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
                                          SubScratch& S, const float* hs, const float* gs, int sub_rows) {
   const int G = gridDim.x, K = p.K, tid = threadIdx.x, nrows = (te - tb) * GEMV_ROWS;
   const int warp = tid >> 5, lane = tid & 31;
+  // Work items: (token, 32 consecutive rows), dealt to the consumer warps in turn; each warp
+  // reduces its item with shuffles and adds the result into the token's shared entry.
+  const int chunks = (nrows + 31) >> 5, items = T * chunks;
   cp_async_wait_all();  // this thread's part of the gain slice
   if (tid < T) {
-    S.my[tid] = 0u;
+    S.mx[tid] = S.my[tid] = 0u;
     S.sum[tid] = 0ull;
+#pragma unroll
+    for (int d = 0; d < ENG_SUB_CAND; ++d) S.cand[tid][d] = 0ull;
   }
   if (tid == 0) S.fallback = 0;
-  // 1. this CTA's max |h| and its candidate sums, a warp per token
-  for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-    const float* hr = hs + t * sub_rows;
-    float m = 0.0f;
-    for (int r = lane; r < nrows; r += 32) m = fmaxf(m, fabsf(hr[r]));
-    m = warp_max(m);
-    long long c[ENG_SUB_CAND];
+  cons_sync();
+  // 1. this CTA's max |h|, then its sums on the candidate grids e_c - d
+  for (int it = warp; it < items; it += ENG_CONS_WARPS) {
+    const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
+    const float m = warp_max(r < nrows ? fabsf(hs[t * sub_rows + r]) : 0.0f);
+    if (lane == 0) atomicMax(&S.mx[t], __float_as_uint(m));
+  }
+  cons_sync();
+  if (tid < T) {
+    const float am = __uint_as_float(S.mx[tid]);
+    S.e[tid] = am > 0.0f ? fixed_point_exponent(__dmul_rn((double)am, (double)am), K) : 0;
+  }
+  cons_sync();
+  if (p.gain != nullptr) {
+    for (int it = warp; it < items; it += ENG_CONS_WARPS) {
+      const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
+      if (S.mx[t] == 0u) continue;
+      const float v = r < nrows ? hs[t * sub_rows + r] : 0.0f;
+      const double d2 = __dmul_rn((double)v, (double)v);
+      double p2e = pow2_f64(S.e[t]);
 #pragma unroll
-    for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] = 0;
-    if (m > 0.0f && p.gain != nullptr) {
-      const int e = fixed_point_exponent(__dmul_rn((double)m, (double)m), K);
-      for (int r = lane; r < nrows; r += 32) {
-        const float v = hr[r];
-#pragma unroll
-        for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] += fixed_sq_term(v, e - d);
+      for (int d = 0; d < ENG_SUB_CAND; ++d) {
+        const long long c = warp_sum_ll(__double2ll_rn(__dmul_rn(d2, p2e)));
+        if (lane == 0) atomicAdd(&S.cand[t][d], (unsigned long long)c);
+        p2e = __dmul_rn(p2e, 0.5);  // the next candidate grid: e - d - 1 (exact)
       }
     }
-#pragma unroll
-    for (int d = 0; d < ENG_SUB_CAND; ++d) c[d] = warp_sum_ll(c[d]);
-    if (lane == 0) {
-      p.pmax[t * G + blockIdx.x] = m;
-      if (p.gain != nullptr)
-#pragma unroll
-        for (int d = 0; d < ENG_SUB_CAND; ++d) p.psum[((long long)t * G + blockIdx.x) * ENG_SUB_CAND + d] = c[d];
-    }
+    cons_sync();
+    if (tid < T * ENG_SUB_CAND)
+      p.psum[((long long)(tid / ENG_SUB_CAND) * G + blockIdx.x) * ENG_SUB_CAND + tid % ENG_SUB_CAND] =
+          (long long)S.cand[tid / ENG_SUB_CAND][tid % ENG_SUB_CAND];
   }
+  if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.mx[tid]);
   if (!grid_step(counters + p.bar_a)) return false;
   // 2. the global max; the sum from the candidates when they cover the global grid
   constexpr int PER = (ENG_MAX_T * ENG_MAX_GRID + ENG_CONS - 1) / ENG_CONS;
@@ -468,8 +483,7 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     const int i = tid + j * ENG_CONS;
     pm[j] = i < T * G ? __ldcg(p.pmax + i) : 0.0f;
   }
-  if (tid < T) S.mx[tid] = 0u;
-  cons_sync();
+  cons_sync();  // this CTA's own max has been published and read: S.mx becomes the global max
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int i = tid + j * ENG_CONS;
@@ -496,13 +510,16 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     }
     cons_sync();
     if (S.fallback) {  // the same decision in every CTA (it follows from the published maxima)
-      for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-        long long c = 0;
-        if (S.mx[t] != 0u)
-          for (int r = lane; r < nrows; r += 32) c += fixed_sq_term(hs[t * sub_rows + r], S.e[t]);
-        c = warp_sum_ll(c);
-        if (lane == 0) p.psum_fb[t * G + blockIdx.x] = c;
+      if (tid < T) S.cand[tid][0] = 0ull;
+      cons_sync();
+      for (int it = warp; it < items; it += ENG_CONS_WARPS) {
+        const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
+        if (S.mx[t] == 0u) continue;
+        const long long c = warp_sum_ll(r < nrows ? fixed_sq_term(hs[t * sub_rows + r], pow2_f64(S.e[t])) : 0ll);
+        if (lane == 0) atomicAdd(&S.cand[t][0], (unsigned long long)c);
       }
+      cons_sync();
+      if (tid < T) p.psum_fb[tid * G + blockIdx.x] = (long long)S.cand[tid][0];
       if (!grid_step(counters + p.bar_fb)) return false;
       if (tid < T) S.sum[tid] = 0ull;
       cons_sync();
@@ -516,14 +533,16 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       S.inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     }
     cons_sync();
-    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-      const float inv = S.inv[t];
-      float m = 0.0f;
-      for (int r = lane; r < nrows; r += 32) m = fmaxf(m, fabsf(__fmul_rn(__fmul_rn(hs[t * sub_rows + r], inv), gs[r])));
-      m = warp_max(m);
-      if (lane == 0) p.pmax2[t * G + blockIdx.x] = m;
+    for (int it = warp; it < items; it += ENG_CONS_WARPS) {
+      const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
+      const float y = r < nrows ? fabsf(__fmul_rn(__fmul_rn(hs[t * sub_rows + r], S.inv[t]), gs[r])) : 0.0f;
+      const float m = warp_max(y);
+      if (lane == 0) atomicMax(&S.my[t], __float_as_uint(m));
     }
+    cons_sync();
+    if (tid < T) p.pmax2[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
     if (!grid_step(counters + p.bar_b)) return false;
+    if (tid < T) S.my[tid] = 0u;
     cons_sync();
     for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.my[i / G], __float_as_uint(__ldcg(p.pmax2 + i)));
     cons_sync();
@@ -534,13 +553,18 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     }
     cons_sync();
   }
-  if (tid < T) S.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(S.my[tid]), 1e-5f));
+  if (tid < T) {
+    S.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(S.my[tid]), 1e-5f));
+    S.sq[tid] = 0;
+  }
   cons_sync();
-  // 4. q of this CTA's rows, four at a time, a warp per token
-  for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-    const float inv = S.inv[t], sc = S.scale[t];
+  // 4. q of this CTA's rows: items of (token, 128 rows), four rows per lane
+  const int qchunks = (nrows + 127) >> 7;
+  for (int it = warp; it < T * qchunks; it += ENG_CONS_WARPS) {
+    const int t = it / qchunks, r = (it - t * qchunks) * 128 + 4 * lane;
     int sum = 0;
-    for (int r = 4 * lane; r < nrows; r += 128) {
+    if (r < nrows) {
+      const float inv = S.inv[t], sc = S.scale[t];
       uint32_t w = 0u;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -554,10 +578,12 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       *reinterpret_cast<uint32_t*>(p.q + (long long)t * K + tb * GEMV_ROWS + r) = w;
     }
     sum = warp_sum_i(sum);
-    if (lane == 0) {
-      atomicAdd(p.sq + t, sum);
-      if (blockIdx.x == 0) p.s[t] = sc;
-    }
+    if (lane == 0) atomicAdd(&S.sq[t], sum);
+  }
+  cons_sync();
+  if (tid < T) {
+    atomicAdd(p.sq + tid, S.sq[tid]);
+    if (blockIdx.x == 0) p.s[tid] = S.scale[tid];
   }
   return true;
 }

@@ -57,12 +57,12 @@ __global__ void __launch_bounds__(256) k_pack_sum(const float* __restrict__ W, l
   __shared__ long long red[32];
   const float M32 = __uint_as_float(sc->max_bits);
   if (M32 == 0.0f) return;
-  const int e = fixed_point_exponent((double)M32, n);
+  const double p2e = pow2_f64(fixed_point_exponent((double)M32, n));
   long long part = 0;
   const long long n4 = n / 4;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(W) + i);
-    part += fixed_abs_term(v.x, e) + fixed_abs_term(v.y, e) + fixed_abs_term(v.z, e) + fixed_abs_term(v.w, e);
+    part += fixed_abs_term(v.x, p2e) + fixed_abs_term(v.y, p2e) + fixed_abs_term(v.z, p2e) + fixed_abs_term(v.w, p2e);
   }
   part = block_reduce(part, red, AddOpLL());
   if (threadIdx.x == 0) atomicAdd(&sc->sum, (unsigned long long)part);

@@ -60,8 +60,9 @@ BN_DEV void quantise_staged_row(float* xs, int K, const float* gain, float eps, 
     if (amax_x > 0.0f) {
       const double M = __dmul_rn((double)amax_x, (double)amax_x);
       const int e = fixed_point_exponent(M, K);
+      const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int k = tid; k < K; k += nt) part += fixed_sq_term(xs[k], e);
+      for (int k = tid; k < K; k += nt) part += fixed_sq_term(xs[k], p2e);
       const long long S = block_reduce(part, redl, AddOpLL());
       ms = fixed_point_mean(S, e, K);
     }
@@ -212,12 +213,13 @@ __global__ void __launch_bounds__(QW_THREADS) k_rmsnorm_quant_warps(const TIn* _
     if (am > 0.0f) {
       const double M = __dmul_rn((double)am, (double)am);
       const int e = fixed_point_exponent(M, K);
+      const double p2e = pow2_f64(e);
       long long part = 0;
 #pragma unroll
       for (int j = 0; j < QW_GROUPS; ++j)
         if (8 * (lane + 32 * (rank + W * j)) < K) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], e);
+          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
         }
       ms = fixed_point_mean(qw_reduce<W>(part, &redl[rr][0], fl, bar, rank, AddOpLL()), e, K);
     }

@@ -55,11 +55,11 @@ __global__ void __launch_bounds__(SHARD_THREADS) k_shard_sumsq(const float* __re
     const float am = amax_g[t];
     long long part = 0;
     if (am > 0.0f) {
-      const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K_total);
+      const double p2e = pow2_f64(fixed_point_exponent(__dmul_rn((double)am, (double)am), K_total));
       const float4* row = reinterpret_cast<const float4*>(h + (long long)t * Ks);
       for (int i = threadIdx.x; i < Ks / 4; i += blockDim.x) {
         const float4 v = row[i];
-        part += fixed_sq_term(v.x, e) + fixed_sq_term(v.y, e) + fixed_sq_term(v.z, e) + fixed_sq_term(v.w, e);
+        part += fixed_sq_term(v.x, p2e) + fixed_sq_term(v.y, p2e) + fixed_sq_term(v.z, p2e) + fixed_sq_term(v.w, p2e);
       }
     }
     part = block_reduce(part, red, AddOpLL());

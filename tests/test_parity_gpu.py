@@ -285,6 +285,38 @@ def test_ffn_block_distributed_sub_norm_without_gain_twice(T, H, I):
     assert tb.device_status() == 0
 
 
+@pytest.mark.parametrize("T", [1, 3])
+def test_ffn_block_distributed_sub_norm_fallback(T):
+    """The grid-wide ffn_sub_norm takes the exact sum from each CTA's candidate grids unless a
+    CTA's max |h| is far below the row's (its candidates then miss the row's grid) -- here
+    the second half of the gate rows has a single non-zero weight each, so the h of those
+    rows is about 2^-6 of the rest and the fallback round runs; bit-exact either way."""
+    H, I = 512, 16512
+    sh = workloads.BlockShape("ffn-fb", hidden=H, n_q=H, n_kv=H, inter=I, act="relu2")
+    d = workloads.block_inputs(sh, T, 77, ffn_only=True)
+    Wg = d["W_gate"].clone()
+    Wg[I // 2:] = 0.0
+    Wg[I // 2:, int(torch.argmax(d["x"][0].float()))] = 0.05  # token 0's largest input: g > 0, relu2(g) > 0
+    pr = {"gate": O.pack_i2s(Wg.numpy()), "up": O.pack_i2s(d["W_up"].numpy()), "down": O.pack_i2s(d["W_down"].numpy())}
+    pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
+    ws = torch.zeros(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
+    ref, mid = O.ffn_block(bf16_to_np(d["x"]), d["g_ffn_norm"].numpy(), pr["gate"], pr["up"],
+                           d["g_ffn_sub_norm"].numpy(), pr["down"], H, I, "relu2", 1e-6, "bf16",
+                           return_intermediates=True)
+    nz = np.abs(mid["h"][0, I // 2:])
+    assert np.max(nz) > 0 and np.max(nz) < np.max(np.abs(mid["h"][0])) * 2.0 ** -4  # far below the row's max
+    off = tb.ffn_workspace_offsets(T, H, I)
+    for _ in range(2):
+        out = tb.ffn_block(d["x"].to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], d["g_ffn_sub_norm"].to(DEV),
+                           pg["down"], I, tb.RELU2, 1e-6, torch.bfloat16, ws=ws)
+        torch.cuda.synchronize()
+        wsn = ws.cpu().numpy()
+        assert np.array_equal(wsn[off[4]:off[4] + T * I].view(np.int8).reshape(T, I), mid["q_h"])
+        assert np.array_equal(wsn[off[6]:off[6] + T * 4].view(np.int32), mid["sum_h"])
+        assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
+    assert tb.device_status() == 0
+
+
 def test_ffn_block_fp32_io():
     out, _, ref, _, dt = run_ffn(2, 384, 512, "silu", seed=5, out_dtype=torch.float32, x_dtype=torch.float32)
     assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
