@@ -114,22 +114,29 @@ __global__ void __launch_bounds__(ATT_THREADS) k_attn_partial(const float* __res
     *reinterpret_cast<float4*>(Qs + j * ATT_KP + d4) =
         __ldg(reinterpret_cast<const float4*>(q + ((long long)t * Hq + h) * ATT_D + d4));
   }
-  for (int i = tid; i < 2 * ATT_CHUNK * (ATT_D / 8); i += ATT_THREADS) {
+  // every thread issues all of its 16-byte loads first (one memory round trip), then widens
+  constexpr int KV_LOADS = 2 * ATT_CHUNK * (ATT_D / 8) / ATT_THREADS;
+  static_assert(KV_LOADS * ATT_THREADS == 2 * ATT_CHUNK * (ATT_D / 8), "whole loads per thread");
+  uint4 w[KV_LOADS];
+#pragma unroll
+  for (int j = 0; j < KV_LOADS; ++j) {
+    const int i = tid + j * ATT_THREADS;
+    const int which = i / (ATT_CHUNK * (ATT_D / 8)), rem = i % (ATT_CHUNK * (ATT_D / 8));
+    const int p = rem / (ATT_D / 8), d8 = (rem % (ATT_D / 8)) * 8;
+    w[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (p < n) w[j] = __ldg(reinterpret_cast<const uint4*>((which ? vc : kc) + ((long long)kv * L_max + c0 + p) * ATT_D + d8));
+  }
+#pragma unroll
+  for (int j = 0; j < KV_LOADS; ++j) {
+    const int i = tid + j * ATT_THREADS;
     const int which = i / (ATT_CHUNK * (ATT_D / 8)), rem = i % (ATT_CHUNK * (ATT_D / 8));
     const int p = rem / (ATT_D / 8), d8 = (rem % (ATT_D / 8)) * 8;
     float* dst = (which ? Vs : Ks) + p * ATT_KP + d8;
-    if (p < n) {
-      const __nv_bfloat16* src = (which ? vc : kc) + ((long long)kv * L_max + c0 + p) * ATT_D + d8;
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        dst[2 * e] = __uint_as_float(ww[e] << 16);
-        dst[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[e] = 0.0f;
+    for (int e = 0; e < 4; ++e) {
+      dst[2 * e] = __uint_as_float(ww[e] << 16);
+      dst[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
     }
   }
   __syncthreads();

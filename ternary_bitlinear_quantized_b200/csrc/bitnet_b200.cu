@@ -142,6 +142,25 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
     if (e != cudaSuccess) return cuda_fail(e, "k_rmsnorm_quant_warps");
     return BITNET_OK;
   }
+  // Long fp32 rows, many of them (the FFN's h at prefill): persistent, double-buffered.
+  if (xt == BITNET_F32 && K % 4 == 0 && 2 * K * 4 <= 227 * 1024 - 1024 && T >= 2 * device_sm_count() && aligned16(x) &&
+      aligned16(q)) {
+    const size_t smem_l = (size_t)2 * K * 4;
+    static std::atomic<int> long_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!long_done[dev & 63].load(std::memory_order_acquire)) {
+      cudaError_t ea = cudaFuncSetAttribute(k_rmsnorm_quant_long, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            227 * 1024 - 1024);
+      if (ea != cudaSuccess) return cuda_fail(ea, "quant attribute (long rows)");
+      long_done[dev & 63].store(1, std::memory_order_release);
+    }
+    const int sms = device_sm_count();
+    cudaError_t el = launch(k_rmsnorm_quant_long, dim3((unsigned)(T < sms ? T : sms)), dim3(QL_THREADS), smem_l, s,
+                            true, reinterpret_cast<const float*>(x), gain, eps, (int)T, (int)K, q, s_x, sum_q);
+    if (el != cudaSuccess) return cuda_fail(el, "k_rmsnorm_quant_long");
+    return BITNET_OK;
+  }
   int threads = (int)((K / 8 + 31) / 32 * 32);
   threads = threads < 128 ? 128 : (threads > 1024 ? 1024 : threads);
   const size_t smem = (size_t)K * sizeof(float);

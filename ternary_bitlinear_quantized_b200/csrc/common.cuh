@@ -123,12 +123,32 @@ BN_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar
                : "memory");
 }
 
+// The same with an L2 cache policy (createpolicy), e.g. evict-first for bytes read once.
+BN_DEV void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+BN_DEV uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // 2-D TMA load of one box of `map` at (x, y) into this CTA's shared memory, completing on
 // barrier `bar` (no multicast).  x * element size must be a multiple of 16 bytes.
 BN_DEV void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
   asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
                ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
                : "memory");
+}
+BN_DEV void tma_load_2d_hint(uint32_t dst, const void* map, int x, int y, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;"
+      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
 }
 
 // 16-byte asynchronous copy global -> shared (both 16-byte aligned), completed by

@@ -150,6 +150,47 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
   quantise_staged_row(xs, K, gain, eps, q + t * K, s_x + t, sum_q + t, vec != 0, red, amax);
 }
 
+// Long fp32 rows (the FFN's h at prefill): one CTA per SM, persistent over rows blockIdx.x,
+// blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with
+// 16-byte cp.async while the current one is reduced, so the row reads stream at the HBM rate
+// instead of waiting behind each row's reduction chain.  The arithmetic is
+// quantise_staged_row's.  K % 4 == 0, rows 16-byte aligned, 2 K floats of shared memory.
+constexpr int QL_THREADS = 1024;
+__global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const float* __restrict__ x,
+                                                                     const float* __restrict__ gain, float eps,
+                                                                     int T, int K, int8_t* __restrict__ q,
+                                                                     float* __restrict__ s_x,
+                                                                     int32_t* __restrict__ sum_q) {
+  extern __shared__ __align__(16) float ql_buf[];  // [2][K]
+  __shared__ long long red[32];
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  auto fetch = [&](long long row, float* dst) {
+    const float* src = x + row * K;
+    for (int i = tid; i < K / 4; i += QL_THREADS) cp_async16(smem_addr(dst + 4 * i), src + 4 * i);
+    cp_async_commit();
+  };
+  long long row = blockIdx.x;
+  if (row < T) fetch(row, ql_buf);
+  for (int it = 0; row < T; ++it, row += gridDim.x) {
+    float* cur = ql_buf + (it & 1) * K;
+    const long long next = row + gridDim.x;
+    if (next < T) {
+      fetch(next, ql_buf + ((it + 1) & 1) * K);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");  // this row's copies (the older group)
+    } else {
+      cp_async_wait_all();
+    }
+    __syncthreads();
+    float am = 0.0f;
+    for (int k = tid; k < K; k += QL_THREADS) am = fmaxf(am, fabsf(cur[k]));
+    am = block_reduce(am, reinterpret_cast<float*>(red), MaxOp());
+    quantise_staged_row(cur, K, gain, eps, q + row * K, s_x + row, sum_q + row, (K % 8) == 0, red, am);
+    __syncthreads();  // the buffer is refilled by the fetch of the next iteration
+  }
+}
+
 // The same arithmetic with W warps per row (W = 1, 2 or 4) and 8 / W rows per 256-thread
 // CTA, for rows of K <= 2048 W values (K a multiple of 8, 16-byte aligned rows).  Lane l of
 // the row's warp `rank` holds elements 8 (l + 32 (rank + W j)) .. +7, j < 8, in registers, so

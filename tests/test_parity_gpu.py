@@ -115,6 +115,8 @@ def test_validate_i2s_matches_oracle(N, K):
     (3, 27648, torch.float32, True, False),
     (2, 28672, torch.bfloat16, True, True),
     (130, 384, torch.bfloat16, True, True),
+    (300, 27648, torch.float32, True, False),   # long fp32 rows, many of them: persistent double-buffered kernel
+    (301, 12288, torch.float32, False, True),
 ])
 def test_quant_bitexact(T, K, dtype, use_gain, outliers):
     x = workloads.activations(T, K, 11, "quant", outliers)
@@ -244,7 +246,7 @@ def run_ffn(T, H, I, act, seed, out_dtype=torch.bfloat16, x_dtype=torch.bfloat16
 @pytest.mark.parametrize("act", ["relu2", "silu"])
 @pytest.mark.parametrize("T,H,I", [(1, 256, 384), (3, 640, 1280), (17, 256, 640), (2, 8192, 512), (10, 1152, 2304),
                                    (64, 512, 768), (130, 384, 1280), (3, 8192, 512), (1, 256, 16512),
-                                   (16, 2048, 1024)])
+                                   (16, 2048, 1024), (300, 256, 9216)])
 def test_ffn_block_parity(act, T, H, I):
     out, ws, ref, mid, dt = run_ffn(T, H, I, act, seed=T + H)
     off = tb.ffn_workspace_offsets(T, H, I)
