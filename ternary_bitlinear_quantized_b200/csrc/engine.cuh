@@ -44,6 +44,7 @@
 namespace bitnet {
 
 constexpr int ENG_CONS_WARPS = 15;  // + 1 producer warp: 16 warps, 4 per SM sub-partition (128 registers each)
+static_assert(ENG_CONS_WARPS == ENG_SLOT_WARPS, "the stage geometry deals slots to the consumer warps");
 constexpr int ENG_CONS = ENG_CONS_WARPS * 32;
 constexpr int ENG_THREADS = ENG_CONS + 32;
 constexpr int ENG_MAX_PHASES = 8;
@@ -619,15 +620,16 @@ struct EngAcc {
   }
 };
 
-// This warp's 64-byte steps of one 16-row tile in a stage: steps t = t0, t0 + 15, .. < S.
+// This warp's 64-byte steps of one 16-row tile in a stage: steps t = t0, t0 + stride, .. < S.
 // Lane (gid, r) holds rows gid and gid + 8 of the tile, bytes 16 r .. 16 r + 15 of each step
 // (the A fragments of mma.sync m16n8k32, one AND per 2-bit field), and the activations of
 // tokens gid (and 8 + gid) -- token T - 1 where those do not exist; those lanes only feed
 // accumulator columns that are never used.  wrow: shared address of row gid's step 0 at
 // byte 16 r; P: row pitch; xa / xb: shared address of the tokens' step 0 (+ 16 r).
 template <int TG>
-BN_DEV void eng_tile_steps(EngAcc<TG>& A, uint32_t wrow, int P, uint32_t xa_s, uint32_t xb_s, int t0, int S) {
-  for (int t = t0; t < S; t += ENG_CONS_WARPS) {
+BN_DEV void eng_tile_steps(EngAcc<TG>& A, uint32_t wrow, int P, uint32_t xa_s, uint32_t xb_s, int t0, int S,
+                           int stride) {
+  for (int t = t0; t < S; t += stride) {
     const uint4 wa = lds128(wrow + 64 * t), wb = lds128(wrow + 8 * P + 64 * t);
     const uint32_t xo = 256u * t;
 #pragma unroll
@@ -740,8 +742,28 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
 
   if (warp == ENG_CONS_WARPS) {
     // ------------------------------------------------------------ producer
-    // Walks the stage order of every product phase (engine_sched.h).  Lane 0 waits for the
-    // slot, sets the expected bytes and issues the copies (no multicast).
+    // First, bulk L2 prefetches (one CTA per slice of the grid) of what the per-phase
+    // quantisations read: every norm gain (immutable) and the raw activation rows of the
+    // phases that do not wait for this launch (L2 is coherent, so a prefetch issued while the
+    // previous kernel may still write them only warms the lines).  They land ahead of the
+    // weight stream, so the quantisations' loads hit L2.
+    if (lane == 0 && blockIdx.x < 8) {
+      for (int pi = 0; pi < a.n_phases; ++pi) {
+        const EngPhase& p = a.ph[pi];
+        const float* g = p.kind == PH_SUBNORM ? nullptr : p.gain;
+        const uint32_t gb = (uint32_t)p.K * 4u;
+        if (g != nullptr && blockIdx.x == (pi & 7)) prefetch_l2_bulk(g, gb);
+        if ((p.kind == PH_QUANT || (ph_is_gemv(p.kind) && p.src == SRC_LOCAL)) && p.wait_barrier < 0 &&
+            blockIdx.x == ((pi + 4) & 7)) {
+          const uint32_t xb = (uint32_t)T * (uint32_t)p.K * (p.x_f32 ? 4u : 2u);
+          prefetch_l2_bulk(p.x, xb);
+        }
+        if (p.kind == PH_GEMV_FFN && p.sub_gain != nullptr && blockIdx.x == (pi & 7))
+          prefetch_l2_bulk(p.sub_gain, (uint32_t)a.ph[pi].t[0].N * 4u);
+      }
+    }
+    // Then walks the stage order of every product phase (engine_sched.h).  Lane 0 waits for
+    // the slot, sets the expected bytes and issues the copies (no multicast).
     int slot = 0, issued = 0;
     uint32_t par = 0;
     bool go = true;  // warp-uniform: false once a wait gave up or the consumers aborted
@@ -938,14 +960,16 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
                   const int S = (cbytes + 63) >> 6;
                   const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (G.CB >> 6));
                   const uint32_t sbase = ring_s + slot * a.slot_bytes + gid * G.CB + 16 * r;
-                  for (int tl = 0; tl < ntg; ++tl) {
-                    int t0 = warp - rot;
-                    if (t0 < 0) t0 += ENG_CONS_WARPS;
-                    eng_tile_steps<TG>(A, sbase + tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S);
-                    rot += S;
-                    while (rot >= ENG_CONS_WARPS) rot -= ENG_CONS_WARPS;
+                  // the stage's tiles go to groups of wpt warps; within a group the steps are
+                  // dealt round-robin, continuing from stage to stage
+                  const int wpt = ENG_CONS_WARPS / G.rs, tl = warp / wpt, wi = warp - tl * wpt;
+                  if (tl < ntg) {
+                    int t0 = wi - rot % wpt;  // rot may come from a phase with another wpt
+                    if (t0 < 0) t0 += wpt;
+                    eng_tile_steps<TG>(A, sbase + tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S, wpt);
                     if (wc == wc1 - 1) A.flush(acc + ((tg0 + tl) * NT + u) * GEMV_ROWS * T, T, gid, r);
                   }
+                  rot = (rot % wpt + S) % wpt;
                   __syncwarp();
                   if (lane == 0) mbar_arrive(empty(slot));
                 }

@@ -3,7 +3,7 @@
 // compiles it as plain C++.
 //
 // A stage (one ring slot) holds weights of ONE tensor: `rs` 16-row tiles x `CB` bytes of each
-// row.  Two modes:
+// row (rs divides the 15 consumer warps; each tile is worked on by 15 / rs of them).  Two modes:
 //   full rows  (CB == RB, the whole row): the tiles' rows are one contiguous byte range of
 //              the I2_S tensor, fetched with one 1-D bulk copy per run of tiles of the same
 //              tensor (large contiguous copies stream at close to the HBM peak);
@@ -30,7 +30,9 @@ constexpr int ENG_BOX_MAX_BYTES = 2048;     // a TMA box row: 256 elements of 8 
 constexpr int ENG_SLOT_MAX = 40 * 1024 + 64;  // bytes of one ring slot at most (a stage + slack)
 constexpr int ENG_ACT_MAX = 72 * 1024;        // shared memory for the staged activations
 constexpr int ENG_STAGE_TARGET = 40 * 1024;  // full-row stages group tiles up to this size
-constexpr int ENG_MAX_RS = 8;                // tiles per full-row stage at most
+constexpr int ENG_MAX_RS = 5;                // tiles per full-row stage at most
+constexpr int ENG_SLOT_WARPS = 15;           // consumer warps sharing a slot; rs divides it, so
+                                             // each tile of a stage gets ENG_SLOT_WARPS / rs warps
 
 struct EngGeom {
   int RB;           // bytes per weight row (K / 4)
@@ -58,10 +60,14 @@ ENG_HD bool eng_plan(int K, int T, int slot_max, int act_max, EngGeom& g) {
   if (16 * RB + 64 <= slot_max && T * eng_x_pitch_for(K) <= act_max) {
     g.full_rows = 1;
     g.CB = RB;
-    int rs = ENG_STAGE_TARGET / (16 * RB);
-    if (rs < 1) rs = 1;
-    if (rs > ENG_MAX_RS) rs = ENG_MAX_RS;
-    while (rs > 1 && 16 * rs * RB + 64 > slot_max) --rs;
+    // tiles per stage: the largest divisor of ENG_SLOT_WARPS (5, 3 or 1) that keeps the
+    // stage within ENG_STAGE_TARGET and the slot
+    int rs = 1;
+    for (int c = ENG_MAX_RS; c > 1; --c)
+      if (ENG_SLOT_WARPS % c == 0 && 16 * c * RB <= ENG_STAGE_TARGET && 16 * c * RB + 64 <= slot_max) {
+        rs = c;
+        break;
+      }
     g.rs = rs;
     g.n_chunks = 1;
     g.ac_chunks = 1;

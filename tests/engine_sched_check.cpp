@@ -33,6 +33,7 @@ int main() {
       if (T * g.x_pitch > ENG_ACT_MAX) fail(K, T, "activations do not fit");
       if (g.full_rows) {
         if (g.CB != RB || g.n_chunks != 1 || g.n_ac != 1 || g.rs < 1 || g.rs > ENG_MAX_RS) fail(K, T, "full-row fields");
+        if (ENG_SLOT_WARPS % g.rs) fail(K, T, "tiles per stage do not divide the consumer warps");
         if (16 * g.rs * RB + 64 > g.slot_bytes) fail(K, T, "full-row slot");
       } else {
         if (g.rs != 1 || g.CB % 64 || g.CB > ENG_BOX_MAX_BYTES || g.CB < 64) fail(K, T, "chunk size");
