@@ -383,6 +383,10 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
           return cuda_fail(cudaErrorInvalidValue, "tensor map (engine weights)");
   }
   qs = (qs + 127) / 128 * 128;
+  // Private accumulator slots per consumer warp when they are small (few tokens): no atomic
+  // contention in the flushes; the epilogue sums the slots.
+  const int acc_priv = acc_ints * ENG_CONS_WARPS * 4 <= 32 * 1024 ? 1 : 0;
+  if (acc_priv) acc_ints *= ENG_CONS_WARPS;
   acc_ints = (acc_ints + 3) / 4 * 4;
   int sub_rows = 0;  // rows of h a CTA keeps for a SUBNORM phase, and their gain
   for (int i = 0; i < a.n_phases; ++i)
@@ -414,6 +418,7 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   a.qs_bytes = qs;
   a.xs_floats = xs;
   a.sub_rows = sub_rows;
+  a.acc_priv = acc_priv;
   const size_t smem =
       1024 + (size_t)slots * slot + 16 * slots + (size_t)acc_ints * 4 + qs + (size_t)xs * 4 + (size_t)sub_floats * 4;
   e = opt_in_smem((const void*)kern, 6 + tg - 1);

@@ -106,7 +106,8 @@ struct alignas(16) EngArgs {
   unsigned* counters;  // ENG_MAX_BARRIERS + 1 words in the workspace (last: exit count)
   int n_slots, slot_bytes, acc_ints, qs_bytes, xs_floats;
   int sub_rows;  // rows of h a CTA keeps for the SUBNORM phase (0: none)
-  int pad_[3];
+  int acc_priv;  // 1: every consumer warp has its own accumulator slots (small T)
+  int pad_[2];
   EngPhase ph[ENG_MAX_PHASES];
 };
 
@@ -476,37 +477,38 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
   }
   if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.mx[tid]);
   if (!grid_step(counters + p.bar_a)) return false;
-  // 2. the global max; the sum from the candidates when they cover the global grid
-  constexpr int PER = (ENG_MAX_T * ENG_MAX_GRID + ENG_CONS - 1) / ENG_CONS;
-  float pm[PER];
-#pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int i = tid + j * ENG_CONS;
-    pm[j] = i < T * G ? __ldcg(p.pmax + i) : 0.0f;
-  }
-  cons_sync();  // this CTA's own max has been published and read: S.mx becomes the global max
-#pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int i = tid + j * ENG_CONS;
-    if (i < T * G) atomicMax(&S.mx[i / G], __float_as_uint(pm[j]));
-  }
-  cons_sync();
-  if (tid < T) {
-    const float am = __uint_as_float(S.mx[tid]);
-    S.e[tid] = am > 0.0f ? fixed_point_exponent(__dmul_rn((double)am, (double)am), K) : 0;
+  // 2. the global max; the sum from the candidates when they cover the global grid.  A warp
+  // per token reads the G published values (independent loads, one round trip) and reduces
+  // them with shuffles: no shared-memory atomics on one address.
+  for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+    float m = 0.0f;
+    for (int c = lane; c < G; c += 32) m = fmaxf(m, __ldcg(p.pmax + t * G + c));
+    m = warp_max(m);
+    if (lane == 0) {
+      S.mx[t] = __float_as_uint(m);
+      S.e[t] = m > 0.0f ? fixed_point_exponent(__dmul_rn((double)m, (double)m), K) : 0;
+    }
   }
   cons_sync();
   if (p.gain != nullptr) {
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int i = tid + j * ENG_CONS;
-      if (i < T * G && pm[j] > 0.0f) {
-        const int t = i / G;
-        const int d = fixed_point_exponent(__dmul_rn((double)pm[j], (double)pm[j]), K) - S.e[t];
-        if (d >= ENG_SUB_CAND)
-          S.fallback = 1;
-        else
-          atomicAdd(&S.sum[t], (unsigned long long)__ldcg(p.psum + (long long)i * ENG_SUB_CAND + d));
+    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+      long long sum = 0;
+      int fb = 0;
+      for (int c = lane; c < G; c += 32) {
+        const float pm = __ldcg(p.pmax + t * G + c);
+        if (pm > 0.0f) {
+          const int d = fixed_point_exponent(__dmul_rn((double)pm, (double)pm), K) - S.e[t];
+          if (d >= ENG_SUB_CAND)
+            fb = 1;
+          else
+            sum += __ldcg(p.psum + ((long long)t * G + c) * ENG_SUB_CAND + d);
+        }
+      }
+      sum = warp_sum_ll(sum);
+      fb = __any_sync(0xffffffffu, fb);
+      if (lane == 0) {
+        S.sum[t] = (unsigned long long)sum;
+        if (fb) S.fallback = 1;
       }
     }
     cons_sync();
@@ -522,9 +524,12 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       cons_sync();
       if (tid < T) p.psum_fb[tid * G + blockIdx.x] = (long long)S.cand[tid][0];
       if (!grid_step(counters + p.bar_fb)) return false;
-      if (tid < T) S.sum[tid] = 0ull;
-      cons_sync();
-      for (int i = tid; i < T * G; i += ENG_CONS) atomicAdd(&S.sum[i / G], (unsigned long long)__ldcg(p.psum_fb + i));
+      for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+        long long sum = 0;
+        for (int c = lane; c < G; c += 32) sum += __ldcg(p.psum_fb + t * G + c);
+        sum = warp_sum_ll(sum);
+        if (lane == 0) S.sum[t] = (unsigned long long)sum;
+      }
       cons_sync();
     }
     // 3. inv and max |y| of this CTA's rows
@@ -543,9 +548,12 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     cons_sync();
     if (tid < T) p.pmax2[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
     if (!grid_step(counters + p.bar_b)) return false;
-    if (tid < T) S.my[tid] = 0u;
-    cons_sync();
-    for (int i = tid; i < T * G; i += ENG_CONS) atomicMax(&S.my[i / G], __float_as_uint(__ldcg(p.pmax2 + i)));
+    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+      float m = 0.0f;
+      for (int c = lane; c < G; c += 32) m = fmaxf(m, __ldcg(p.pmax2 + t * G + c));
+      m = warp_max(m);
+      if (lane == 0) S.my[t] = __float_as_uint(m);
+    }
     cons_sync();
   } else {
     if (tid < T) {
@@ -604,8 +612,10 @@ struct EngAcc {
         for (int i = 0; i < 4; ++i) f[tg][g][i] = 0;
   }
   // Combine the fields exactly (field g's sums are multiples of 4^(3-g)) and add this warp's
-  // share into the tile's shared accumulator at[row * T + tok]; then restart.
-  BN_DEV void flush(int* at, int T, int gid, int r) {
+  // share into the tile's shared accumulator at[row * T + tok] -- with an atomic add into the
+  // slot all warps share, or (priv) a plain add into this warp's own slot, which the
+  // epilogue sums (no contention of 15 warps on the same words); then restart.
+  BN_DEV void flush(int* at, int T, int gid, int r, bool priv) {
 #pragma unroll
     for (int tg = 0; tg < TG; ++tg)
 #pragma unroll
@@ -613,7 +623,11 @@ struct EngAcc {
         const int tok = tg * 8 + 2 * r + (i & 1);
         if (tok < T) {
           const int v = (f[tg][0][i] >> 6) + (f[tg][1][i] >> 4) + (f[tg][2][i] >> 2) + f[tg][3][i];
-          atomicAdd(at + (gid + ((i & 2) ? 8 : 0)) * T + tok, v);
+          int* dst = at + (gid + ((i & 2) ? 8 : 0)) * T + tok;
+          if (priv)
+            *dst += v;
+          else
+            atomicAdd(dst, v);
         }
       }
     zero();
@@ -850,7 +864,6 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
     pdl_wait();  // activations and workspace belong to the previous kernel until now
     int slot = 0;       // ring position of the next stage
     uint32_t par = 0;   // and the phase parity of its barriers
-    int rot = 0;        // round-robin position of the 64-byte steps over the warps
     // The SUBNORM phases accumulate sum_q with atomics: clear it before any CTA can get
     // there (the grid barrier of the gate/up phase comes first).
     if (blockIdx.x == 0 && threadIdx.x < T)
@@ -917,7 +930,10 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
           }
         }
       }
-      for (int i = threadIdx.x; i < nt * NT * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
+      // Accumulators: [tile][tensor][16 rows][T], or with private warp slots (a.acc_priv)
+      // [tile][tensor][warp][16 rows][T].
+      const int aw = a.acc_priv ? ENG_CONS_WARPS : 1;
+      for (int i = threadIdx.x; i < nt * NT * aw * GEMV_ROWS * T; i += ENG_CONS) acc[i] = 0;
       if (p.pmax != nullptr && p.sub_gain != nullptr) {
         // the SUBNORM phase's gain for this CTA's rows, fetched while the products run
         for (int i = threadIdx.x; i < nt * GEMV_ROWS / 4; i += ENG_CONS)
@@ -932,6 +948,11 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         const uint32_t ring_s = smem_addr(ring);
         EngAcc<TG> A;
         A.zero();
+        // the stage's tiles go to groups of wpt warps (per phase constants); within a group the
+        // steps are dealt round-robin, continuing from stage to stage
+        const int wpt = ENG_CONS_WARPS / G.rs, my_tl = warp / wpt, my_wi = warp - my_tl * wpt;
+        const int S_full = (G.CB + 63) >> 6;  // steps of a whole chunk
+        int rot = 0;
         // A warp whose wait gives up stops waiting and computing but keeps walking the stage
         // order, so that every consumer thread meets the same named barriers; the decision
         // to leave is taken together at the next one (barrier.red.or).
@@ -956,20 +977,19 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
               for (int wc = wc0; wc < wc1; ++wc) {
                 if (ok && !mbar_wait_bounded(full(slot), par)) ok = false;
                 if (ok) {
-                  const int cbytes = min(G.CB, G.RB - wc * G.CB);
-                  const int S = (cbytes + 63) >> 6;
+                  const int S = wc < G.n_chunks - 1 ? S_full : (G.RB - wc * G.CB + 63) >> 6;
                   const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (G.CB >> 6));
                   const uint32_t sbase = ring_s + slot * a.slot_bytes + gid * G.CB + 16 * r;
-                  // the stage's tiles go to groups of wpt warps; within a group the steps are
-                  // dealt round-robin, continuing from stage to stage
-                  const int wpt = ENG_CONS_WARPS / G.rs, tl = warp / wpt, wi = warp - tl * wpt;
-                  if (tl < ntg) {
-                    int t0 = wi - rot % wpt;  // rot may come from a phase with another wpt
+                  if (my_tl < ntg) {
+                    int t0 = my_wi - rot;
                     if (t0 < 0) t0 += wpt;
-                    eng_tile_steps<TG>(A, sbase + tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S, wpt);
-                    if (wc == wc1 - 1) A.flush(acc + ((tg0 + tl) * NT + u) * GEMV_ROWS * T, T, gid, r);
+                    eng_tile_steps<TG>(A, sbase + my_tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S, wpt);
+                    if (wc == wc1 - 1)
+                      A.flush(acc + (((tg0 + my_tl) * NT + u) * aw + (a.acc_priv ? warp : 0)) * GEMV_ROWS * T, T,
+                              gid, r, a.acc_priv != 0);
                   }
-                  rot = (rot % wpt + S) % wpt;
+                  rot += S;
+                  while (rot >= wpt) rot -= wpt;
                   __syncwarp();
                   if (lane == 0) mbar_arrive(empty(slot));
                 }
@@ -997,13 +1017,18 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         const int sq = local ? s_loc_sq[t] : __ldcg(p.sq + t);
         // s_x may be absent when only the int32 accumulators are asked for (no float output).
         const float sx = local ? s_loc_s[t] : (p.s != nullptr ? __ldcg(p.s + t) : 1.0f);
-        const int* at = acc + tl2 * NT * GEMV_ROWS * T;
-        const int accA = at[row * T + t] - sq;
+        const int* at = acc + tl2 * NT * aw * GEMV_ROWS * T;
+        int sumA = 0, sumU = 0;
+        for (int w = 0; w < aw; ++w) {
+          sumA += at[(w * GEMV_ROWS + row) * T + t];
+          if (NT == 2) sumU += at[((aw + w) * GEMV_ROWS + row) * T + t];
+        }
+        const int accA = sumA - sq;
         const float betaA = s_beta[pi][ti];
         const float vA = dequant(accA, __fdiv_rn(betaA, sx));
         if (NT == 2) {
           const float betaU = s_beta[pi][1];
-          const int accU = at[(GEMV_ROWS + row) * T + t] - sq;
+          const int accU = sumU - sq;
           const float vU = dequant(accU, __fdiv_rn(betaU, sx));
           const float hv = ffn_act(vA, vU, p.act);
           p.h[(long long)t * N + n] = hv;
