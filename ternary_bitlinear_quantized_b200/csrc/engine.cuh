@@ -362,12 +362,12 @@ BN_DEV void quant_row(const void* xrow, int x_f32, int K, const float* gain, flo
 }
 
 // ------------------------------------------------------------------ grid barriers
+// Arrival is a release add at GPU scope by one thread after the CTA barrier: the barrier
+// orders the other consumer threads' writes before it, and release is cumulative, so a CTA
+// whose acquire load sees the count also sees those writes (no separate full fence).
 BN_DEV void grid_arrive(unsigned* ctr) {
   cons_sync();  // every consumer thread of this CTA has written its outputs
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
-  }
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
 BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
@@ -386,7 +386,8 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
         break;
       }
     }
-    __threadfence();
+    // the acquire load that saw the count orders this thread's later reads; the named
+    // barrier that follows every wait passes that on to the other consumer threads
   }
   return ok;
 }
@@ -478,32 +479,39 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
   if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.mx[tid]);
   if (!grid_step(counters + p.bar_a)) return false;
   // 2. the global max; the sum from the candidates when they cover the global grid.  A warp
-  // per token reads the G published values (independent loads, one round trip) and reduces
-  // them with shuffles: no shared-memory atomics on one address.
+  // per token loads the G published maxima at once (unrolled, predicated: one round trip),
+  // reduces them with shuffles, then loads the matching candidate sums at once (a second
+  // round trip).  No shared-memory atomics on one address.
+  constexpr int GPL = ENG_MAX_GRID / 32;  // published values per lane at most
   for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-    float m = 0.0f;
-    for (int c = lane; c < G; c += 32) m = fmaxf(m, __ldcg(p.pmax + t * G + c));
-    m = warp_max(m);
-    if (lane == 0) {
-      S.mx[t] = __float_as_uint(m);
-      S.e[t] = m > 0.0f ? fixed_point_exponent(__dmul_rn((double)m, (double)m), K) : 0;
+    float pm[GPL];
+#pragma unroll
+    for (int j = 0; j < GPL; ++j) {
+      const int c = lane + 32 * j;
+      pm[j] = c < G ? __ldcg(p.pmax + t * G + c) : 0.0f;
     }
-  }
-  cons_sync();
-  if (p.gain != nullptr) {
-    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-      long long sum = 0;
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < GPL; ++j) m = fmaxf(m, pm[j]);
+    m = warp_max(m);
+    const int e = m > 0.0f ? fixed_point_exponent(__dmul_rn((double)m, (double)m), K) : 0;
+    if (p.gain != nullptr) {
+      long long v[GPL];
       int fb = 0;
-      for (int c = lane; c < G; c += 32) {
-        const float pm = __ldcg(p.pmax + t * G + c);
-        if (pm > 0.0f) {
-          const int d = fixed_point_exponent(__dmul_rn((double)pm, (double)pm), K) - S.e[t];
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) {
+        v[j] = 0;
+        if (pm[j] > 0.0f) {
+          const int d = fixed_point_exponent(__dmul_rn((double)pm[j], (double)pm[j]), K) - e;
           if (d >= ENG_SUB_CAND)
             fb = 1;
           else
-            sum += __ldcg(p.psum + ((long long)t * G + c) * ENG_SUB_CAND + d);
+            v[j] = __ldcg(p.psum + ((long long)t * G + lane + 32 * j) * ENG_SUB_CAND + d);
         }
       }
+      long long sum = 0;
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) sum += v[j];
       sum = warp_sum_ll(sum);
       fb = __any_sync(0xffffffffu, fb);
       if (lane == 0) {
@@ -511,7 +519,13 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
         if (fb) S.fallback = 1;
       }
     }
-    cons_sync();
+    if (lane == 0) {
+      S.mx[t] = __float_as_uint(m);
+      S.e[t] = e;
+    }
+  }
+  cons_sync();
+  if (p.gain != nullptr) {
     if (S.fallback) {  // the same decision in every CTA (it follows from the published maxima)
       if (tid < T) S.cand[tid][0] = 0ull;
       cons_sync();
@@ -549,8 +563,15 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     if (tid < T) p.pmax2[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
     if (!grid_step(counters + p.bar_b)) return false;
     for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+      float pm[GPL];
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) {
+        const int c = lane + 32 * j;
+        pm[j] = c < G ? __ldcg(p.pmax2 + t * G + c) : 0.0f;
+      }
       float m = 0.0f;
-      for (int c = lane; c < G; c += 32) m = fmaxf(m, __ldcg(p.pmax2 + t * G + c));
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) m = fmaxf(m, pm[j]);
       m = warp_max(m);
       if (lane == 0) S.my[t] = __float_as_uint(m);
     }
