@@ -208,6 +208,30 @@ BN_DEV long long fixed_sq_term(float v, double p2e) {
 }
 BN_DEV long long fixed_abs_term(float v, double p2e) { return __double2ll_rn(__dmul_rn((double)fabsf(v), p2e)); }
 
+// Rounding to an integer without a conversion instruction (conversions issue at a quarter of
+// the fp64 add rate): adding 1.5 * 2^52 to a double x with |x| < 2^51 leaves rint(x) -- the
+// addition rounds to the nearest integer, ties to even -- in the low bits of the significand.
+BN_DEV long long rint_i64_small(double x) {
+  return __double_as_longlong(__dadd_rn(x, 6755399441055744.0)) - 0x4338000000000000ll;
+}
+// The sums' n terms are each below 2^(62 - ceil_log2(n)), hence below 2^51 once n > 1024.
+constexpr long long kFixedSmallMinN = 1025;
+template <bool SMALL>
+BN_DEV long long fixed_sq_term_t(float v, double p2e) {
+  if (!SMALL) return fixed_sq_term(v, p2e);
+  const double d = (double)v;
+  return rint_i64_small(__dmul_rn(__dmul_rn(d, d), p2e));
+}
+
+// int8 code of an activation: clamp(rint(p), -128, 127), ties to even, for the fp32 product
+// p = y * s (NaN gives 0, as the conversion instruction does).  Clamping first keeps |p| below
+// 2^22, where adding 1.5 * 2^23 rounds p to an integer in the low significand bits.
+BN_DEV int quant_code(float p) {
+  const float c = fminf(fmaxf(p, -128.0f), 127.0f);
+  const int q = __float_as_int(__fadd_rn(c, 12582912.0f)) - 0x4B400000;
+  return p == p ? q : 0;
+}
+
 // ---------------------------------------------------------------- reductions
 BN_DEV float warp_max(float v) {
 #pragma unroll

@@ -236,11 +236,21 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
       const double p2e = pow2_f64(e);
       long long part = 0;
+      if (K >= kFixedSmallMinN) {
 #pragma unroll
-      for (int j = 0; j < ENG_REG_GROUPS; ++j) {
-        if (8 * (tid + ENG_CONS * j) < K) {
+        for (int j = 0; j < ENG_REG_GROUPS; ++j) {
+          if (8 * (tid + ENG_CONS * j) < K) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
+            for (int i = 0; i < 8; ++i) part += fixed_sq_term_t<true>(v[j][i], p2e);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < ENG_REG_GROUPS; ++j) {
+          if (8 * (tid + ENG_CONS * j) < K) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
+          }
         }
       }
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
@@ -268,8 +278,7 @@ __device__ __noinline__ void quant_row_regs(const void* xrow, int x_f32, int K, 
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int qv = __float2int_rn(__fmul_rn(v[j][i], s));
-        qv = min(127, max(-128, qv));
+        int qv = quant_code(__fmul_rn(v[j][i], s));
         sum += qv;
         w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
       }
@@ -320,7 +329,10 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
       const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
       const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term(xs[kk], p2e);
+      if (K >= kFixedSmallMinN)
+        for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term_t<true>(xs[kk], p2e);
+      else
+        for (int kk = tid; kk < K; kk += ENG_CONS) part += fixed_sq_term(xs[kk], p2e);
       ms = fixed_point_mean(cons_sum_i64(part, R), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
@@ -338,8 +350,7 @@ __device__ __noinline__ void quant_row_staged(const void* xrow, int x_f32, int K
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      int qv = __float2int_rn(__fmul_rn(xs[kk + i], s));
-      qv = min(127, max(-128, qv));
+      int qv = quant_code(__fmul_rn(xs[kk + i], s));
       sum += qv;
       w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
     }
@@ -466,7 +477,8 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       double p2e = pow2_f64(S.e[t]);
 #pragma unroll
       for (int d = 0; d < ENG_SUB_CAND; ++d) {
-        const long long c = warp_sum_ll(__double2ll_rn(__dmul_rn(d2, p2e)));
+        const double x2 = __dmul_rn(d2, p2e);
+        const long long c = warp_sum_ll(K >= kFixedSmallMinN ? rint_i64_small(x2) : __double2ll_rn(x2));
         if (lane == 0) atomicAdd(&S.cand[t][d], (unsigned long long)c);
         p2e = __dmul_rn(p2e, 0.5);  // the next candidate grid: e - d - 1 (exact)
       }
@@ -600,8 +612,7 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       for (int k = 0; k < 4; ++k) {
         float y = hs[t * sub_rows + r + k];
         if (p.gain != nullptr) y = __fmul_rn(__fmul_rn(y, inv), gs[r + k]);
-        int qv = __float2int_rn(__fmul_rn(y, sc));
-        qv = min(127, max(-128, qv));
+        int qv = quant_code(__fmul_rn(y, sc));
         sum += qv;
         w |= (uint32_t)(qv & 0xFF) << (8 * k);
       }
@@ -653,6 +664,22 @@ struct EngAcc {
       }
     zero();
   }
+  // The same for one token (T = 1): lanes with r == 0 hold token 0 of rows gid (i = 0) and
+  // gid + 8 (i = 2).
+  BN_DEV void flush1(int* at, int gid, int r, bool priv) {
+    if (r == 0) {
+      const int v0 = (f[0][0][0] >> 6) + (f[0][1][0] >> 4) + (f[0][2][0] >> 2) + f[0][3][0];
+      const int v2 = (f[0][0][2] >> 6) + (f[0][1][2] >> 4) + (f[0][2][2] >> 2) + f[0][3][2];
+      if (priv) {
+        at[gid] += v0;
+        at[gid + 8] += v2;
+      } else {
+        atomicAdd(at + gid, v0);
+        atomicAdd(at + gid + 8, v2);
+      }
+    }
+    zero();
+  }
 };
 
 // This warp's 64-byte steps of one 16-row tile in a stage: steps t = t0, t0 + stride, .. < S.
@@ -681,6 +708,49 @@ BN_DEV void eng_tile_steps(EngAcc<TG>& A, uint32_t wrow, int P, uint32_t xa_s, u
         mma_u8s8(A.f[TG - 1][g], a4, a5, a6, a7, x1.z, x1.w);
       }
     }
+  }
+}
+
+// The stages of one activation chunk range [wc0, wc1) of a product phase whose stages hold one
+// 16-row tile of one tensor each (rs = 1): for every (tile, tensor) in order, its chunks; the
+// warp's steps of the chunk are t0, t0 + 15, .. (t0 rotating from stage to stage); after the
+// tile's last chunk the flush into `at`, which then advances by at_step.  A flat loop with the
+// chunk width CBC fixed at compile time where it is known (0: run-time CBr), and the one-token
+// flush for T1: the general loop nest ran about a quarter slower per stage.
+template <int TG, int CBC, bool T1>
+BN_DEV void eng_flat_stages(EngAcc<TG>& A, int n_tu, int wc0, int wc1, int n_chunks, int CBr, int RB, uint32_t ring_s,
+                            int slot_bytes, int n_slots, uint32_t full0, uint32_t empty0, uint32_t xa0, uint32_t xb0,
+                            int* at, int at_step, int T, bool priv, int warp, int gid, int r, int lane, int& slot,
+                            uint32_t& par, int& rot, bool& ok) {
+  const int CB = CBC ? CBC : CBr;
+  const int S_full = (CB + 63) >> 6, S_last = (RB - (n_chunks - 1) * CB + 63) >> 6;
+  const uint32_t row_off = gid * CB + 16 * r;
+  for (int i = 0; i < n_tu; ++i) {
+    for (int wc = wc0; wc < wc1; ++wc) {
+      if (ok && !mbar_wait_bounded(full0 + 8u * slot, par)) ok = false;
+      if (ok) {
+        const int S = wc < n_chunks - 1 ? S_full : S_last;
+        const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (CB >> 6));
+        int t0 = warp - rot;
+        if (t0 < 0) t0 += ENG_CONS_WARPS;
+        eng_tile_steps<TG>(A, ring_s + slot * slot_bytes + row_off, CB, xa0 + xoff, xb0 + xoff, t0, S, ENG_CONS_WARPS);
+        if (wc == wc1 - 1) {
+          if (T1)
+            A.flush1(at, gid, r, priv);
+          else
+            A.flush(at, T, gid, r, priv);
+        }
+        rot += S;
+        while (rot >= ENG_CONS_WARPS) rot -= ENG_CONS_WARPS;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+      }
+      if (++slot == n_slots) {
+        slot = 0;
+        par ^= 1u;
+      }
+    }
+    at += at_step;
   }
 }
 
@@ -821,7 +891,14 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
                 ok = s_abort == 0 && mbar_wait_bounded(empty(slot), par ^ 1u);
                 if (ok) {
                   const uint32_t dst = smem_addr(ring + slot * a.slot_bytes);
-                  if (G.full_rows) {
+                  if (G.full_rows && ntg == 1) {
+                    // one tile: one contiguous copy of its rows
+                    int ti, n0, nr;
+                    locate(p, tb + tg0, ti, n0, nr);
+                    const uint32_t bytes = (uint32_t)nr * G.RB;
+                    mbar_arrive_expect_tx(full(slot), bytes);
+                    bulk_g2s(dst, p.t[NT == 2 ? u : ti].packed + (long long)n0 * G.RB, bytes, full(slot));
+                  } else if (G.full_rows) {
                     // runs of consecutive tiles of the same tensor: one contiguous copy each
                     uint32_t bytes = 0;
                     for (int pass = 0; pass < 2; ++pass) {
@@ -969,52 +1046,80 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
         const uint32_t ring_s = smem_addr(ring);
         EngAcc<TG> A;
         A.zero();
-        // the stage's tiles go to groups of wpt warps (per phase constants); within a group the
-        // steps are dealt round-robin, continuing from stage to stage
-        const int wpt = ENG_CONS_WARPS / G.rs, my_tl = warp / wpt, my_wi = warp - my_tl * wpt;
-        const int S_full = (G.CB + 63) >> 6;  // steps of a whole chunk
+        // The stage's tiles go to groups of wpt warps (per phase constants); within a group the
+        // steps are dealt round-robin, continuing from stage to stage.  The stage loop's
+        // parameters are taken out of the shared descriptors once.
+        const int CB = G.CB, RB = G.RB, n_chunks = G.n_chunks, rs = G.rs, n_ac = G.n_ac, ac_chunks = G.ac_chunks;
+        const int n_slots = a.n_slots, slot_bytes = a.slot_bytes;
+        const bool priv = a.acc_priv != 0;
+        const uint32_t full0 = full(0), empty0 = empty(0);
+        const int wpt = ENG_CONS_WARPS / rs, my_tl = warp / wpt, my_wi = warp - my_tl * wpt;
+        const int S_full = (CB + 63) >> 6;  // steps of a whole chunk
+        int* const acc_w = acc + (priv ? warp : 0) * GEMV_ROWS * T;
         int rot = 0;
         // A warp whose wait gives up stops waiting and computing but keeps walking the stage
         // order, so that every consumer thread meets the same named barriers; the decision
         // to leave is taken together at the next one (barrier.red.or).
         bool ok = true;
-        for (int ac = 0; ac < G.n_ac; ++ac) {
-          const int wc0 = ac * G.ac_chunks, wc1 = min(G.n_chunks, wc0 + G.ac_chunks);
+        for (int ac = 0; ac < n_ac; ++ac) {
+          const int wc0 = ac * ac_chunks, wc1 = min(n_chunks, wc0 + ac_chunks);
           if (!local) {
             // the previous chunk's readers are done, then stage this chunk
             if (named_sync_or(1, ENG_CONS, !ok)) {
               ok = false;
               break;
             }
-            eng_stage_acts(p.q, p.K, T, 4 * wc0 * G.CB, min(p.K, 4 * wc1 * G.CB), qs, G.x_pitch);
+            eng_stage_acts(p.q, p.K, T, 4 * wc0 * CB, min(p.K, 4 * wc1 * CB), qs, G.x_pitch);
           }
           if (named_sync_or(1, ENG_CONS, !ok)) {
             ok = false;
             break;
           }
-          for (int tg0 = 0; tg0 < nt; tg0 += G.rs) {
-            const int ntg = min(G.rs, nt - tg0);
+          if (rs == 1) {
+            const int at_step = aw * GEMV_ROWS * T;
+            if (TG == 1 && T == 1) {
+              if (CB == 2048)
+                eng_flat_stages<TG, 2048, true>(A, nt * NT, wc0, wc1, n_chunks, CB, RB, ring_s, slot_bytes, n_slots, full0,
+                                                empty0, xa0, xb0, acc_w, at_step, T, priv, warp, gid, r, lane, slot, par,
+                                                rot, ok);
+              else
+                eng_flat_stages<TG, 0, true>(A, nt * NT, wc0, wc1, n_chunks, CB, RB, ring_s, slot_bytes, n_slots, full0,
+                                             empty0, xa0, xb0, acc_w, at_step, T, priv, warp, gid, r, lane, slot, par, rot,
+                                             ok);
+            } else {
+              if (CB == 2048)
+                eng_flat_stages<TG, 2048, false>(A, nt * NT, wc0, wc1, n_chunks, CB, RB, ring_s, slot_bytes, n_slots, full0,
+                                                 empty0, xa0, xb0, acc_w, at_step, T, priv, warp, gid, r, lane, slot, par,
+                                                 rot, ok);
+              else
+                eng_flat_stages<TG, 0, false>(A, nt * NT, wc0, wc1, n_chunks, CB, RB, ring_s, slot_bytes, n_slots, full0,
+                                              empty0, xa0, xb0, acc_w, at_step, T, priv, warp, gid, r, lane, slot, par, rot,
+                                              ok);
+            }
+            continue;
+          }
+          for (int tg0 = 0; tg0 < nt; tg0 += rs) {
+            const int ntg = min(rs, nt - tg0);
             for (int u = 0; u < NT; ++u) {
               for (int wc = wc0; wc < wc1; ++wc) {
-                if (ok && !mbar_wait_bounded(full(slot), par)) ok = false;
+                if (ok && !mbar_wait_bounded(full0 + 8u * slot, par)) ok = false;
                 if (ok) {
-                  const int S = wc < G.n_chunks - 1 ? S_full : (G.RB - wc * G.CB + 63) >> 6;
-                  const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (G.CB >> 6));
-                  const uint32_t sbase = ring_s + slot * a.slot_bytes + gid * G.CB + 16 * r;
+                  const int S = wc < n_chunks - 1 ? S_full : (RB - wc * CB + 63) >> 6;
+                  const uint32_t xoff = 256u * (uint32_t)((wc - wc0) * (CB >> 6));
+                  const uint32_t sbase = ring_s + slot * slot_bytes + gid * CB + 16 * r;
                   if (my_tl < ntg) {
                     int t0 = my_wi - rot;
                     if (t0 < 0) t0 += wpt;
-                    eng_tile_steps<TG>(A, sbase + my_tl * GEMV_ROWS * G.CB, G.CB, xa0 + xoff, xb0 + xoff, t0, S, wpt);
+                    eng_tile_steps<TG>(A, sbase + my_tl * GEMV_ROWS * CB, CB, xa0 + xoff, xb0 + xoff, t0, S, wpt);
                     if (wc == wc1 - 1)
-                      A.flush(acc + (((tg0 + my_tl) * NT + u) * aw + (a.acc_priv ? warp : 0)) * GEMV_ROWS * T, T,
-                              gid, r, a.acc_priv != 0);
+                      A.flush(acc_w + ((tg0 + my_tl) * NT + u) * aw * GEMV_ROWS * T, T, gid, r, priv);
                   }
                   rot += S;
                   while (rot >= wpt) rot -= wpt;
                   __syncwarp();
-                  if (lane == 0) mbar_arrive(empty(slot));
+                  if (lane == 0) mbar_arrive(empty0 + 8u * slot);
                 }
-                if (++slot == a.n_slots) {
+                if (++slot == n_slots) {
                   slot = 0;
                   par ^= 1u;
                 }

@@ -62,7 +62,10 @@ BN_DEV void quantise_staged_row(float* xs, int K, const float* gain, float eps, 
       const int e = fixed_point_exponent(M, K);
       const double p2e = pow2_f64(e);
       long long part = 0;
-      for (int k = tid; k < K; k += nt) part += fixed_sq_term(xs[k], p2e);
+      if (K >= kFixedSmallMinN)
+        for (int k = tid; k < K; k += nt) part += fixed_sq_term_t<true>(xs[k], p2e);
+      else
+        for (int k = tid; k < K; k += nt) part += fixed_sq_term(xs[k], p2e);
       const long long S = block_reduce(part, redl, AddOpLL());
       ms = fixed_point_mean(S, e, K);
     }
@@ -87,8 +90,7 @@ BN_DEV void quantise_staged_row(float* xs, int K, const float* gain, float eps, 
         uint32_t packed = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          int v = __float2int_rn(__fmul_rn(xs[k + 4 * h + j], s));
-          v = min(127, max(-128, v));
+          int v = quant_code(__fmul_rn(xs[k + 4 * h + j], s));
           sum += v;
           packed |= (uint32_t)(v & 0xFF) << (8 * j);
         }
@@ -98,8 +100,7 @@ BN_DEV void quantise_staged_row(float* xs, int K, const float* gain, float eps, 
     }
   } else {
     for (int k = tid; k < K; k += nt) {
-      int v = __float2int_rn(__fmul_rn(xs[k], s));
-      v = min(127, max(-128, v));
+      int v = quant_code(__fmul_rn(xs[k], s));
       sum += v;
       qrow[k] = (int8_t)v;
     }
@@ -256,12 +257,21 @@ __global__ void __launch_bounds__(QW_THREADS) k_rmsnorm_quant_warps(const TIn* _
       const int e = fixed_point_exponent(M, K);
       const double p2e = pow2_f64(e);
       long long part = 0;
+      if (K >= kFixedSmallMinN) {
 #pragma unroll
-      for (int j = 0; j < QW_GROUPS; ++j)
-        if (8 * (lane + 32 * (rank + W * j)) < K) {
+        for (int j = 0; j < QW_GROUPS; ++j)
+          if (8 * (lane + 32 * (rank + W * j)) < K) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
-        }
+            for (int i = 0; i < 8; ++i) part += fixed_sq_term_t<true>(v[j][i], p2e);
+          }
+      } else {
+#pragma unroll
+        for (int j = 0; j < QW_GROUPS; ++j)
+          if (8 * (lane + 32 * (rank + W * j)) < K) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) part += fixed_sq_term(v[j][i], p2e);
+          }
+      }
       ms = fixed_point_mean(qw_reduce<W>(part, &redl[rr][0], fl, bar, rank, AddOpLL()), e, K);
     }
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
@@ -292,8 +302,7 @@ __global__ void __launch_bounds__(QW_THREADS) k_rmsnorm_quant_warps(const TIn* _
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int qv = __float2int_rn(__fmul_rn(v[j][i], s));
-        qv = min(127, max(-128, qv));
+        int qv = quant_code(__fmul_rn(v[j][i], s));
         sum += qv;
         w[i >> 2] |= (uint32_t)(qv & 0xFF) << (8 * (i & 3));
       }

@@ -57,9 +57,17 @@ __global__ void __launch_bounds__(SHARD_THREADS) k_shard_sumsq(const float* __re
     if (am > 0.0f) {
       const double p2e = pow2_f64(fixed_point_exponent(__dmul_rn((double)am, (double)am), K_total));
       const float4* row = reinterpret_cast<const float4*>(h + (long long)t * Ks);
-      for (int i = threadIdx.x; i < Ks / 4; i += blockDim.x) {
-        const float4 v = row[i];
-        part += fixed_sq_term(v.x, p2e) + fixed_sq_term(v.y, p2e) + fixed_sq_term(v.z, p2e) + fixed_sq_term(v.w, p2e);
+      if (K_total >= kFixedSmallMinN) {
+        for (int i = threadIdx.x; i < Ks / 4; i += blockDim.x) {
+          const float4 v = row[i];
+          part += fixed_sq_term_t<true>(v.x, p2e) + fixed_sq_term_t<true>(v.y, p2e) + fixed_sq_term_t<true>(v.z, p2e) +
+                  fixed_sq_term_t<true>(v.w, p2e);
+        }
+      } else {
+        for (int i = threadIdx.x; i < Ks / 4; i += blockDim.x) {
+          const float4 v = row[i];
+          part += fixed_sq_term(v.x, p2e) + fixed_sq_term(v.y, p2e) + fixed_sq_term(v.z, p2e) + fixed_sq_term(v.w, p2e);
+        }
       }
     }
     part = block_reduce(part, red, AddOpLL());
@@ -135,8 +143,7 @@ __global__ void __launch_bounds__(SHARD_THREADS) k_shard_quant(const float* __re
       uint32_t w = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        int qv = __float2int_rn(__fmul_rn(y[j], s));
-        qv = min(127, max(-128, qv));
+        int qv = quant_code(__fmul_rn(y[j], s));
         sum += qv;
         w |= (uint32_t)(qv & 0xFF) << (8 * j);
       }
