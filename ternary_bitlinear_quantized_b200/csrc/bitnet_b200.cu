@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <algorithm>
 #include <string>
 
 #include "common.cuh"
@@ -351,6 +352,50 @@ static bool make_map_u64(CUtensorMap* m, const void* base, uint64_t N, uint64_t 
 }
 
 // Launch the engine over the phases in `a` (a.T, a.eps, a.n_phases, a.ph, a.counters set).
+// Balanced tile split (see EngPhase::balanced) of the product phases that run back to back
+// from the first one up to the first QUANT or SUBNORM phase (no grid-wide wait between them
+// blocks a CTA for long): each phase's n_tiles mod G extra tiles go to the CTAs with the least
+// work so far, heaviest phases first, work counted in weight bytes per tile.  A SUBNORM phase
+// takes the split of the phase before it (it reduces the rows that phase produced).
+static void balance_tiles(EngArgs& a, int grid) {
+  int first = 0;
+  while (first < a.n_phases && !ph_is_gemv(a.ph[first].kind)) ++first;
+  int last = first;
+  while (last < a.n_phases && ph_is_gemv(a.ph[last].kind)) ++last;  // [first, last)
+  if (last - first >= 2 && grid >= 2 && grid <= ENG_MAX_GRID) {
+    int order[ENG_MAX_PHASES], n = 0;
+    for (int i = first; i < last; ++i) order[n++] = i;
+    auto tile_bytes = [&](const EngPhase& p) {
+      return (long long)(p.kind == PH_GEMV_FFN ? 2 : 1) * GEMV_ROWS * (p.K / 4);
+    };
+    for (int i = 1; i < n; ++i)  // heaviest tiles first (stable)
+      for (int j = i; j > 0 && tile_bytes(a.ph[order[j]]) > tile_bytes(a.ph[order[j - 1]]); --j) {
+        const int t = order[j];
+        order[j] = order[j - 1];
+        order[j - 1] = t;
+      }
+    long long load[ENG_MAX_GRID];
+    int idx[ENG_MAX_GRID];
+    for (int c = 0; c < grid; ++c) load[c] = 0;
+    for (int k = 0; k < n; ++k) {
+      EngPhase& p = a.ph[order[k]];
+      const int base = p.n_tiles / grid, extra = p.n_tiles % grid;
+      for (int c = 0; c < grid; ++c) idx[c] = c;
+      std::stable_sort(idx, idx + grid, [&](int x, int y) { return load[x] < load[y]; });
+      p.balanced = 1;
+      memset(p.xmask, 0, sizeof(p.xmask));
+      for (int j = 0; j < extra; ++j) p.xmask[idx[j] >> 5] |= 1u << (idx[j] & 31);
+      for (int c = 0; c < grid; ++c)
+        load[c] += tile_bytes(p) * (base + (int)((p.xmask[c >> 5] >> (c & 31)) & 1u));
+    }
+  }
+  for (int i = 1; i < a.n_phases; ++i)
+    if (a.ph[i].kind == PH_SUBNORM && ph_is_gemv(a.ph[i - 1].kind)) {
+      a.ph[i].balanced = a.ph[i - 1].balanced;
+      memcpy(a.ph[i].xmask, a.ph[i - 1].xmask, sizeof(a.ph[i].xmask));
+    }
+}
+
 static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
   static_assert(sizeof(EngArgs) % 16 == 0, "EngArgs is copied with 16-byte loads");
   const int sms = device_sm_count();
@@ -360,6 +405,7 @@ static bitnet_status enqueue_engine(EngArgs& a, cudaStream_t s) {
     if (ph_is_gemv(a.ph[i].kind) && a.ph[i].n_tiles > max_tiles) max_tiles = a.ph[i].n_tiles;
   const int gmax = sms < ENG_MAX_GRID ? sms : ENG_MAX_GRID;  // per-CTA partials are sized for ENG_MAX_GRID
   const int grid = multi ? gmax : (max_tiles < gmax ? max_tiles : gmax);
+  balance_tiles(a, grid);
   int acc_ints = 0, qs = 0, xs = 0, slot = 0;
   EngMaps maps;
   memset(&maps, 0, sizeof(maps));

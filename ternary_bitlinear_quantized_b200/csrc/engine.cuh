@@ -90,6 +90,12 @@ struct EngPhase {
   float* pmax2;
   const float* sub_gain;
   int bar_a, bar_b, bar_fb;
+  // Tile split over the grid: CTA c owns tiles [start(c), start(c + 1)); by default
+  // start(c) = floor(c n_tiles / G).  Balanced split (balanced = 1): every CTA gets
+  // floor(n_tiles / G) tiles plus one where bit c of xmask is set, so that the host can
+  // spread the remainders of consecutive phases over different CTAs.
+  int balanced;
+  uint32_t xmask[ENG_MAX_GRID / 32];
   EngGeom g;  // stage geometry of a product phase (engine_sched.h)
 };
 
@@ -834,8 +840,17 @@ __global__ void __launch_bounds__(ENG_THREADS, 1) k_engine(const __grid_constant
   pdl_launch_dependents();
 
   auto tile_range = [&](const EngPhase& p, int& tb, int& te) {
-    tb = (int)((long long)blockIdx.x * p.n_tiles / gridDim.x);
-    te = (int)((long long)(blockIdx.x + 1) * p.n_tiles / gridDim.x);
+    if (p.balanced) {
+      const int base = p.n_tiles / (int)gridDim.x, c = blockIdx.x;
+      int below = 0;
+      for (int w = 0; w < (c >> 5); ++w) below += __popc(p.xmask[w]);
+      below += __popc(p.xmask[c >> 5] & ((1u << (c & 31)) - 1u));
+      tb = c * base + below;
+      te = tb + base + (int)((p.xmask[c >> 5] >> (c & 31)) & 1u);
+    } else {
+      tb = (int)((long long)blockIdx.x * p.n_tiles / gridDim.x);
+      te = (int)((long long)(blockIdx.x + 1) * p.n_tiles / gridDim.x);
+    }
   };
   auto locate = [&](const EngPhase& p, int tile, int& ti, int& n0, int& nrows) {
     ti = 0;
