@@ -412,6 +412,7 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 // ------------------------------------------------------------------ distributed sub-norm
 // Per-token scratch of the SUBNORM phase in shared memory.
 constexpr int ENG_SUB_CAND = 8;  // candidate grids per CTA: local exponent e_c, e_c - 1, .., e_c - 7
+static_assert(ENG_SUB_CAND == 8, "the candidate sums are reduced by a three-level lane split");
 struct SubScratch {
   unsigned mx[ENG_MAX_T];  // max |h|: this CTA's, then the row's (non-negative floats as bits)
   unsigned my[ENG_MAX_T];  // max |y|
@@ -481,13 +482,37 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       const float v = r < nrows ? hs[t * sub_rows + r] : 0.0f;
       const double d2 = __dmul_rn((double)v, (double)v);
       double p2e = pow2_f64(S.e[t]);
+      long long c[ENG_SUB_CAND];
 #pragma unroll
       for (int d = 0; d < ENG_SUB_CAND; ++d) {
         const double x2 = __dmul_rn(d2, p2e);
-        const long long c = warp_sum_ll(K >= kFixedSmallMinN ? rint_i64_small(x2) : __double2ll_rn(x2));
-        if (lane == 0) atomicAdd(&S.cand[t][d], (unsigned long long)c);
+        c[d] = K >= kFixedSmallMinN ? rint_i64_small(x2) : __double2ll_rn(x2);
         p2e = __dmul_rn(p2e, 0.5);  // the next candidate grid: e - d - 1 (exact)
       }
+      // The 8 warp sums at once (reduce-scatter): at each of the first three steps a lane keeps
+      // the half of its values selected by one lane bit and adds its partner's copy of that
+      // half; lane l then holds candidate (l >> 2) & 7 summed over 8 lanes, and two more steps
+      // finish the sums (9 exchanges instead of 40).
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool hi = lane & 16;
+        const long long send = hi ? c[i] : c[i + 4], keep = hi ? c[i + 4] : c[i];
+        c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bool hi = lane & 8;
+        const long long send = hi ? c[i] : c[i + 2], keep = hi ? c[i + 2] : c[i];
+        c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+      {
+        const bool hi = lane & 4;
+        const long long send = hi ? c[0] : c[1], keep = hi ? c[1] : c[0];
+        c[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      c[0] += __shfl_xor_sync(0xffffffffu, c[0], 2);
+      c[0] += __shfl_xor_sync(0xffffffffu, c[0], 1);
+      if ((lane & 3) == 0) atomicAdd(&S.cand[t][(lane >> 2) & 7], (unsigned long long)c[0]);
     }
     cons_sync();
     if (tid < T * ENG_SUB_CAND)
