@@ -144,8 +144,8 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
     return BITNET_OK;
   }
   // Long fp32 rows, many of them (the FFN's h at prefill): persistent, double-buffered.
-  if (xt == BITNET_F32 && K % 4 == 0 && 2 * K * 4 <= 227 * 1024 - 1024 && T >= 2 * device_sm_count() && aligned16(x) &&
-      aligned16(q)) {
+  if (xt == BITNET_F32 && K % 4 == 0 && 2 * K * 4 <= 227 * 1024 - 1024 && K <= QL_THREADS * QL_MAXJ &&
+      T >= 2 * device_sm_count() && aligned16(x) && aligned16(q)) {
     const size_t smem_l = (size_t)2 * K * 4;
     static std::atomic<int> long_done[64] = {};
     int dev = 0;
@@ -227,7 +227,8 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
         best_bn = bn;
       }
     }
-    a.BN = best_bn;
+    // The FFN product runs with the roles swapped (128 tokens as the MMA's M): BN = 128.
+    a.BN = ffn ? TC_BM : best_bn;
   }
   a.n_tensors = g.n_tensors;
   a.out_dtype = g.out_dtype;
@@ -251,7 +252,9 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
   }
   a.m_tiles = mt;
   a.tok_tiles = (g.T + a.BN - 1) / a.BN;
-  const uint32_t stage_bytes = (uint32_t)((NT * TC_BM * TC_BK + a.BN * TC_BK + NT * TC_BM * 32 + 1023) / 1024 * 1024);
+  // TMA stages (B tile + packed weights) after TC_A_BUFS expanded weight buffers.
+  const uint32_t stage_bytes = (uint32_t)((a.BN * TC_BK + NT * TC_BM * 32 + 1023) / 1024 * 1024);
+  const uint32_t abuf_bytes = (uint32_t)(TC_A_BUFS * NT * TC_BM * TC_BK);
   int dev = 0, max_optin = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -259,11 +262,11 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
   void (*kern)(const TcMaps, const TcArgs) = ffn ? k_gemm_tc<true> : k_gemm_tc<false>;
   cudaError_t e = cudaFuncGetAttributes(&fa, (const void*)kern);
   if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc attributes");
-  int stages = (int)((max_optin - (int)fa.sharedSizeBytes - 1024 - 256) / stage_bytes);
+  int stages = (int)((max_optin - (int)fa.sharedSizeBytes - 1024 - 256 - (int)abuf_bytes) / (int)stage_bytes);
   if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
   if (stages < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_gemm_tc stages");
   a.stages = stages;
-  const size_t smem = (size_t)stages * stage_bytes + 1024 + 256;
+  const size_t smem = (size_t)abuf_bytes + (size_t)stages * stage_bytes + 1024 + 256;
   e = opt_in_smem((const void*)kern, 4 + (ffn ? 1 : 0));
   if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc attribute");
   const int total = a.m_tiles * a.tok_tiles;

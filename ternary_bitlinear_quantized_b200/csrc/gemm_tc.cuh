@@ -40,7 +40,8 @@ constexpr int TC_EPI_WARPS = 4;      // warps 0-3
 constexpr int TC_TMA_WARP = 4;
 constexpr int TC_MMA_WARP = 5;
 constexpr int TC_EXP_WARP0 = 6;
-constexpr int TC_MAX_STAGES = 6;
+constexpr int TC_MAX_STAGES = 8;
+constexpr int TC_A_BUFS = 2;        // expanded weight tiles in flight (decoupled from the TMA stages)
 
 struct TcTensor {
   const uint8_t* packed;
@@ -117,6 +118,13 @@ BN_DEV uint64_t umma_desc_sw128(uint32_t saddr) {
 BN_DEV uint32_t umma_idesc_i8(int bn) {
   return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
 }
+// The FFN's product with the roles swapped: D s32 [128 tokens x 256], A s8 (activations, M = 128
+// tokens), B u8 (the gate and up codes of one 128-row tile, stacked: N = 256).  One instruction
+// then covers both tensors, and at twice the N each instruction runs long enough for the single
+// issuing thread to keep the tensor pipe fed.
+BN_DEV uint32_t umma_idesc_i8_ffn() {
+  return (2u << 4) | (1u << 7) | (0u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
 
 template <bool FFN>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant__ TcMaps maps, const TcArgs a) {
@@ -130,27 +138,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BN = a.BN, S = a.stages, KB = a.K / TC_BK;
-  // Stage layout (1024-byte aligned): A tiles [NT][128 x 128], B tile [BN x 128], packed [NT][128 x 32].
+  // Shared layout (1024-byte aligned): TC_A_BUFS expanded weight buffers [NT][128 x 128],
+  // then S TMA stages of B tile [BN x 128] + packed [NT][128 x 32].  The TMA stages run deeper
+  // than the expanded buffers: the operand loads stay ahead of the expansion by S stages.
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
   const uint32_t a_bytes = TC_BM * TC_BK, b_bytes = (uint32_t)BN * TC_BK, p_bytes = TC_BM * 32;
-  const uint32_t stage_bytes = (NT * a_bytes + b_bytes + NT * p_bytes + 1023u) & ~1023u;
-  auto sA = [&](int s, int u) { return base + s * stage_bytes + u * a_bytes; };
-  auto sB = [&](int s) { return base + s * stage_bytes + NT * a_bytes; };
-  auto sP = [&](int s, int u) { return base + s * stage_bytes + NT * a_bytes + b_bytes + u * p_bytes; };
-  const uint32_t bars = base + S * stage_bytes;
+  const uint32_t stage_bytes = (b_bytes + NT * p_bytes + 1023u) & ~1023u;
+  const uint32_t tma0 = base + TC_A_BUFS * NT * a_bytes;
+  auto sA = [&](int xb, int u) { return base + (xb * NT + u) * a_bytes; };
+  auto sB = [&](int s) { return tma0 + s * stage_bytes; };
+  auto sP = [&](int s, int u) { return tma0 + s * stage_bytes + b_bytes + u * p_bytes; };
+  const uint32_t bars = tma0 + S * stage_bytes;
   auto full_tma = [&](int s) { return bars + 8u * s; };
-  auto full_a = [&](int s) { return bars + 8u * (TC_MAX_STAGES + s); };
-  auto empty = [&](int s) { return bars + 8u * (2 * TC_MAX_STAGES + s); };
-  auto tm_full = [&](int b) { return bars + 8u * (3 * TC_MAX_STAGES + b); };
-  auto tm_empty = [&](int b) { return bars + 8u * (3 * TC_MAX_STAGES + 2 + b); };
-  const uint32_t mma_done = bars + 8u * (3 * TC_MAX_STAGES + 4);  // final commit after an abort
+  auto empty = [&](int s) { return bars + 8u * (TC_MAX_STAGES + s); };
+  auto full_a = [&](int xb) { return bars + 8u * (2 * TC_MAX_STAGES + xb); };
+  auto tm_full = [&](int b) { return bars + 8u * (2 * TC_MAX_STAGES + 2 * TC_A_BUFS + b); };
+  auto tm_empty = [&](int b) { return bars + 8u * (2 * TC_MAX_STAGES + 2 * TC_A_BUFS + 2 + b); };
+  const uint32_t mma_done = bars + 8u * (2 * TC_MAX_STAGES + 2 * TC_A_BUFS + 4);  // final commit after an abort
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_tma(s), 1);
-      mbar_init(full_a(s), TC_EXP_WARPS * 32);
       mbar_init(empty(s), 1);
     }
+    for (int xb = 0; xb < TC_A_BUFS; ++xb) mbar_init(full_a(xb), TC_EXP_WARPS * 32);
     for (int b = 0; b < 2; ++b) {
       mbar_init(tm_full(b), 1);
       mbar_init(tm_empty(b), 128);
@@ -211,8 +222,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     int it = 0;
     for (int lin = blockIdx.x; lin < total && !s_abort; lin += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb, ++it) {
-        const int s = it % S;
-        if (!mbar_wait_bounded(full_tma(s), (it / S) & 1)) {
+        const int s = it % S, xb = it % TC_A_BUFS;  // TMA stage, expanded buffer
+        // Buffer xb was last read by the MMAs of iteration it - TC_A_BUFS, whose commit also
+        // completes that iteration's stage barrier: wait for that phase (the MMAs cannot be
+        // more than one iteration ahead of this one, so the parity cannot alias).
+        const int pv = it - TC_A_BUFS;
+        if (!mbar_wait_bounded(full_tma(s), (it / S) & 1) ||
+            (pv >= 0 && !mbar_wait_bounded(empty(pv % S), (pv / S) & 1))) {
           s_abort = 1;
           break;
         }
@@ -224,7 +240,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
           const uint32_t pa = sP(s, u) + r * 32;
           const uint4 f0 = lds128(pa + sw), f1 = lds128(pa + (16u - sw));
           const uint4 w0 = sw ? f1 : f0, w1 = sw ? f0 : f1;
-          const uint32_t rowa = sA(s, u) + r * 128;
+          const uint32_t rowa = sA(xb, u) + r * 128;
 #pragma unroll
           for (int gg = 0; gg < 2; ++gg) {
             const int g = 2 * h + gg;
@@ -242,49 +258,61 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
           }
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-        mbar_arrive(full_a(s));
+        mbar_arrive(full_a(xb));
       }
     }
   } else if (warp == TC_MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = umma_idesc_i8(BN);
-    int it = 0, tcount = 0;
-    for (int lin = blockIdx.x; lin < total && !s_abort; lin += gridDim.x, ++tcount) {
-      const int ab = tcount & 1;
+    // One thread runs the whole loop (stage and buffer indices and their barrier parities kept
+    // incrementally): between two k-blocks it has only the waits and a commit to do, so the
+    // tensor pipe's queue does not run dry.
+    if (lane == 0) {
+      const uint32_t idesc = FFN ? umma_idesc_i8_ffn() : umma_idesc_i8(BN);
+      int s = 0, xb = 0, tcount = 0;
+      uint32_t ph_s = 0, ph_x = 0;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(tm_empty(ab), ((tcount >> 1) & 1) ^ 1);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        s_abort = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t dcol = tmem + (uint32_t)(ab * NT * BN);
-      for (int kb = 0; kb < KB; ++kb, ++it) {
-        const int s = it % S;
-        if (lane == 0) {
-          ok = mbar_wait_bounded(full_a(s), (it / S) & 1) && mbar_wait_bounded(full_tma(s), (it / S) & 1);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          s_abort = 1;
+      for (int lin = blockIdx.x; ok && lin < total && !s_abort; lin += gridDim.x, ++tcount) {
+        const int ab = tcount & 1;
+        if (!mbar_wait_bounded(tm_empty(ab), ((tcount >> 1) & 1) ^ 1)) {
+          ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = umma_desc_sw128(sB(s) + 32 * kk);
-#pragma unroll
-            for (int u = 0; u < NT; ++u)
-              umma_i8(dcol + u * BN, umma_desc_sw128(sA(s, u) + 32 * kk), bdesc, idesc, (kb | kk) ? 1u : 0u);
+        const uint32_t dcol = tmem + (uint32_t)(ab * NT * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(full_a(xb), ph_x) || !mbar_wait_bounded(full_tma(s), ph_s)) {
+            ok = false;
+            break;
           }
-          umma_commit(empty(s));
+          tc_fence_after();
+          if (FFN) {
+            // D[token][gate row | up row]: A = the activation tile, B = both expanded code tiles
+            // (sA(xb, 0) and sA(xb, 1) are adjacent: 256 rows in the same swizzled layout).
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_i8(dcol, umma_desc_sw128(sB(s) + 32 * kk), umma_desc_sw128(sA(xb, 0) + 32 * kk), idesc,
+                      (kb | kk) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_i8(dcol, umma_desc_sw128(sA(xb, 0) + 32 * kk), umma_desc_sw128(sB(s) + 32 * kk), idesc,
+                      (kb | kk) ? 1u : 0u);
+          }
+          umma_commit(empty(s));  // frees the TMA stage and (to the expanders) the expanded buffer
           if (kb == KB - 1) umma_commit(tm_full(ab));
+          if (++s == S) {
+            s = 0;
+            ph_s ^= 1u;
+          }
+          if (++xb == TC_A_BUFS) {
+            xb = 0;
+            ph_x ^= 1u;
+          }
         }
-        __syncwarp();
       }
+      if (!ok) s_abort = 1;
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (warps 0-3)
     pdl_wait();
@@ -300,6 +328,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
       const int ab = tcount & 1;
       const int N = a.t[ti].N;
       const long long row_bytes = a.K >> 2;
+      if (FFN) {
+        // Swapped roles: TMEM lane = token tok0 + et, columns [0, 128) gate and [128, 256) up of
+        // weight rows m0 .. m0 + 127; this thread writes 16 consecutive h values per chunk.
+        const int t = tok0 + et;
+        const bool tok_ok = t < a.T;
+        const float sx = (tok_ok && a.s_x != nullptr) ? __ldg(a.s_x + t) : 1.0f;
+        const int sq = tok_ok ? __ldg(a.sum_q + t) : 0;
+        const float betaG = __ldg(reinterpret_cast<const float*>(a.t[0].packed + (long long)N * row_bytes));
+        const float betaU = __ldg(reinterpret_cast<const float*>(a.t[1].packed + (long long)N * row_bytes));
+        const float fG = __fdiv_rn(betaG, sx), fU = __fdiv_rn(betaU, sx);
+        const bool ok = mbar_wait_bounded(tm_full(ab), (tcount >> 1) & 1);
+        tc_fence_after();
+        for (int c0 = 0; ok && c0 < TC_BM; c0 += 16) {
+          uint32_t vg[16], vu[16];
+          tmem_ld16(tmem + lane_base + (uint32_t)(ab * 256 + c0), vg);
+          tmem_ld16(tmem + lane_base + (uint32_t)(ab * 256 + TC_BM + c0), vu);
+          tmem_wait_ld();
+          if (c0 + 16 >= TC_BM) {
+            tc_fence_before();
+            mbar_arrive(tm_empty(ab));  // accumulator may be overwritten now
+          }
+          if (!tok_ok || m0 + c0 >= N) continue;
+          float hv[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            hv[j] = ffn_act(dequant((int)vg[j] - sq, fG), dequant((int)vu[j] - sq, fU), a.act);
+          float4* dst = reinterpret_cast<float4*>(a.h + (long long)t * N + m0 + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_float4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
+        }
+        if (named_sync_or(1, 128, !ok)) {
+          s_abort = 1;
+          break;
+        }
+        continue;
+      }
       // Per-token factors of this tile: beta / s_x and the activation sum.
       for (int j = et; j < BN; j += 128) {
         const int t = tok0 + j;

@@ -154,9 +154,13 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
 // Long fp32 rows (the FFN's h at prefill): one CTA per SM, persistent over rows blockIdx.x,
 // blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with
 // 16-byte cp.async while the current one is reduced, so the row reads stream at the HBM rate
-// instead of waiting behind each row's reduction chain.  The arithmetic is
-// quantise_staged_row's.  K % 4 == 0, rows 16-byte aligned, 2 K floats of shared memory.
+// instead of waiting behind each row's reduction chain.  Thread i owns elements
+// i + QL_THREADS j; its gain values stay in registers for all rows (reading them from L2 per
+// row put a memory round trip behind every element of the y pass).  The arithmetic is
+// quantise_staged_row's.  K % 4 == 0, K <= QL_THREADS QL_MAXJ, rows 16-byte aligned,
+// 2 K floats of shared memory.
 constexpr int QL_THREADS = 1024;
+constexpr int QL_MAXJ = 28;  // K <= 28672
 __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const float* __restrict__ x,
                                                                      const float* __restrict__ gain, float eps,
                                                                      int T, int K, int8_t* __restrict__ q,
@@ -165,6 +169,12 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
   extern __shared__ __align__(16) float ql_buf[];  // [2][K]
   __shared__ long long red[32];
   const int tid = threadIdx.x;
+  float gr[QL_MAXJ];
+#pragma unroll
+  for (int j = 0; j < QL_MAXJ; ++j) {
+    const int k = tid + QL_THREADS * j;
+    gr[j] = (gain != nullptr && k < K) ? __ldg(gain + k) : 0.0f;
+  }
   pdl_launch_dependents();
   pdl_wait();
   auto fetch = [&](long long row, float* dst) {
@@ -185,9 +195,64 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
     }
     __syncthreads();
     float am = 0.0f;
-    for (int k = tid; k < K; k += QL_THREADS) am = fmaxf(am, fabsf(cur[k]));
+#pragma unroll
+    for (int j = 0; j < QL_MAXJ; ++j) {
+      const int k = tid + QL_THREADS * j;
+      if (k < K) am = fmaxf(am, fabsf(cur[k]));
+    }
     am = block_reduce(am, reinterpret_cast<float*>(red), MaxOp());
-    quantise_staged_row(cur, K, gain, eps, q + row * K, s_x + row, sum_q + row, (K % 8) == 0, red, am);
+    float a = am;
+    if (gain != nullptr) {
+      float ms = 0.0f;
+      if (am > 0.0f) {
+        const int e = fixed_point_exponent(__dmul_rn((double)am, (double)am), K);
+        const double p2e = pow2_f64(e);
+        long long part = 0;
+        if (K >= kFixedSmallMinN) {
+#pragma unroll
+          for (int j = 0; j < QL_MAXJ; ++j) {
+            const int k = tid + QL_THREADS * j;
+            if (k < K) part += fixed_sq_term_t<true>(cur[k], p2e);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < QL_MAXJ; ++j) {
+            const int k = tid + QL_THREADS * j;
+            if (k < K) part += fixed_sq_term(cur[k], p2e);
+          }
+        }
+        ms = fixed_point_mean(block_reduce(part, red, AddOpLL()), e, K);
+      }
+      const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+      float ay = 0.0f;
+#pragma unroll
+      for (int j = 0; j < QL_MAXJ; ++j) {
+        const int k = tid + QL_THREADS * j;
+        if (k < K) {
+          const float y = __fmul_rn(__fmul_rn(cur[k], inv), gr[j]);
+          cur[k] = y;
+          ay = fmaxf(ay, fabsf(y));
+        }
+      }
+      a = block_reduce(ay, reinterpret_cast<float*>(red), MaxOp());
+    }
+    const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+    int sum = 0;
+    int8_t* qrow = q + row * K;
+#pragma unroll
+    for (int j = 0; j < QL_MAXJ; ++j) {
+      const int k = tid + QL_THREADS * j;
+      if (k < K) {
+        const int v = quant_code(__fmul_rn(cur[k], s));
+        sum += v;
+        qrow[k] = (int8_t)v;
+      }
+    }
+    sum = block_reduce(sum, reinterpret_cast<int*>(red), AddOpI());
+    if (tid == 0) {
+      s_x[row] = s;
+      sum_q[row] = sum;
+    }
     __syncthreads();  // the buffer is refilled by the fetch of the next iteration
   }
 }
