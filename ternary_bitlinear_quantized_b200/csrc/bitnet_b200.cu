@@ -264,7 +264,7 @@ static bitnet_status enqueue_gemm_tc(const GemvArgs& g, bool ffn, cudaStream_t s
   if (e != cudaSuccess) return cuda_fail(e, "k_gemm_tc attributes");
   int stages = (int)((max_optin - (int)fa.sharedSizeBytes - 1024 - 256 - (int)abuf_bytes) / (int)stage_bytes);
   if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
-  if (stages < 2) return cuda_fail(cudaErrorInvalidConfiguration, "k_gemm_tc stages");
+  if (stages < TC_A_BUFS) return cuda_fail(cudaErrorInvalidConfiguration, "k_gemm_tc stages");
   a.stages = stages;
   const size_t smem = (size_t)abuf_bytes + (size_t)stages * stage_bytes + 1024 + 256;
   e = opt_in_smem((const void*)kern, 4 + (ffn ? 1 : 0));

@@ -35,13 +35,16 @@ namespace bitnet {
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 128;
 constexpr int TC_EXP_WARPS = 8;     // warps 6-13: two threads per tile row
+constexpr int TC_EXP_PARTS = TC_EXP_WARPS * 32 / 128;  // threads per tile row
+constexpr int TC_FPP = 4 / TC_EXP_PARTS;               // 2-bit fields per thread
+static_assert(TC_EXP_PARTS * TC_FPP == 4, "the expander threads split a row's four fields");
 constexpr int TC_THREADS = (6 + TC_EXP_WARPS) * 32;
 constexpr int TC_EPI_WARPS = 4;      // warps 0-3
 constexpr int TC_TMA_WARP = 4;
 constexpr int TC_MMA_WARP = 5;
 constexpr int TC_EXP_WARP0 = 6;
 constexpr int TC_MAX_STAGES = 8;
-constexpr int TC_A_BUFS = 2;        // expanded weight tiles in flight (decoupled from the TMA stages)
+constexpr int TC_A_BUFS = 3;        // expanded weight tiles in flight (decoupled from the TMA stages)
 
 struct TcTensor {
   const uint8_t* packed;
@@ -224,8 +227,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = it % S, xb = it % TC_A_BUFS;  // TMA stage, expanded buffer
         // Buffer xb was last read by the MMAs of iteration it - TC_A_BUFS, whose commit also
-        // completes that iteration's stage barrier: wait for that phase (the MMAs cannot be
-        // more than one iteration ahead of this one, so the parity cannot alias).
+        // completes that iteration's stage barrier: wait for that phase.  The MMAs are at most
+        // at iteration it - 1, and the stage's next completion after it - TC_A_BUFS is at
+        // it - TC_A_BUFS + S >= it (S >= TC_A_BUFS), so the parity cannot alias.
         const int pv = it - TC_A_BUFS;
         if (!mbar_wait_bounded(full_tma(s), (it / S) & 1) ||
             (pv >= 0 && !mbar_wait_bounded(empty(pv % S), (pv / S) & 1))) {
@@ -242,8 +246,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
           const uint4 w0 = sw ? f1 : f0, w1 = sw ? f0 : f1;
           const uint32_t rowa = sA(xb, u) + r * 128;
 #pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            const int g = 2 * h + gg;
+          for (int gg = 0; gg < TC_FPP; ++gg) {
+            const int g = TC_FPP * h + gg;
             const int sh = 6 - 2 * g;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
