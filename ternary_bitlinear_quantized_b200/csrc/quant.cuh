@@ -152,9 +152,9 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
 }
 
 // Long fp32 rows (the FFN's h at prefill): one CTA per SM, persistent over rows blockIdx.x,
-// blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with
-// 16-byte cp.async while the current one is reduced, so the row reads stream at the HBM rate
-// instead of waiting behind each row's reduction chain.  Thread i owns elements
+// blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with one
+// bulk copy (completing on the buffer's mbarrier) while the current one is reduced, so the
+// row reads stream at the HBM rate instead of waiting behind each row's reduction chain.  Thread i owns elements
 // i + QL_THREADS j; its gain values stay in registers for all rows (reading them from L2 per
 // row put a memory round trip behind every element of the y pass).  The arithmetic is
 // quantise_staged_row's.  K % 4 == 0, K <= QL_THREADS QL_MAXJ, rows 16-byte aligned,
@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
                                                                      int32_t* __restrict__ sum_q) {
   extern __shared__ __align__(16) float ql_buf[];  // [2][K]
   __shared__ long long red[32];
+  __shared__ __align__(8) unsigned long long ql_bar[2];  // one per row buffer: its bulk copy landed
+  volatile __shared__ int ql_abort;
   const int tid = threadIdx.x;
   float gr[QL_MAXJ];
 #pragma unroll
@@ -175,25 +177,38 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
     const int k = tid + QL_THREADS * j;
     gr[j] = (gain != nullptr && k < K) ? __ldg(gain + k) : 0.0f;
   }
+  if (tid == 0) {
+    mbar_init(smem_addr(&ql_bar[0]), 1);
+    mbar_init(smem_addr(&ql_bar[1]), 1);
+    ql_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
   pdl_launch_dependents();
   pdl_wait();
-  auto fetch = [&](long long row, float* dst) {
-    const float* src = x + row * K;
-    for (int i = tid; i < K / 4; i += QL_THREADS) cp_async16(smem_addr(dst + 4 * i), src + 4 * i);
-    cp_async_commit();
+  // One bulk copy per row (thread 0), completing on the buffer's barrier.
+  const uint32_t row_bytes = (uint32_t)K * 4u;
+  auto fetch = [&](long long row, int b) {
+    mbar_arrive_expect_tx(smem_addr(&ql_bar[b]), row_bytes);
+    bulk_g2s(smem_addr(ql_buf + b * K), x + row * K, row_bytes, smem_addr(&ql_bar[b]));
   };
   long long row = blockIdx.x;
-  if (row < T) fetch(row, ql_buf);
+  int issued = 0;
+  if (tid == 0 && row < T) {
+    fetch(row, 0);
+    issued = 1;
+  }
   for (int it = 0; row < T; ++it, row += gridDim.x) {
-    float* cur = ql_buf + (it & 1) * K;
+    const int b = it & 1;
+    float* cur = ql_buf + b * K;
     const long long next = row + gridDim.x;
-    if (next < T) {
-      fetch(next, ql_buf + ((it + 1) & 1) * K);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");  // this row's copies (the older group)
-    } else {
-      cp_async_wait_all();
+    if (tid == 0 && next < T) {  // the other buffer was released by the barrier at the end of it - 1
+      fetch(next, b ^ 1);
+      ++issued;
     }
+    if (!mbar_wait_bounded(smem_addr(&ql_bar[b]), (uint32_t)((it >> 1) & 1))) ql_abort = 1;
     __syncthreads();
+    if (ql_abort) break;
     float am = 0.0f;
 #pragma unroll
     for (int j = 0; j < QL_MAXJ; ++j) {
@@ -253,8 +268,12 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
       s_x[row] = s;
       sum_q[row] = sum;
     }
-    __syncthreads();  // the buffer is refilled by the fetch of the next iteration
+    fence_proxy_async_smem();  // this thread's y writes ordered before the buffer's next bulk copy
+    __syncthreads();           // the buffer is refilled by the fetch of the next iteration
   }
+  // After a wait gave up, the copies still in flight land (fixed limit) before the CTA exits.
+  if (tid == 0 && ql_abort)
+    for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k) mbar_drain(smem_addr(&ql_bar[k & 1]), (uint32_t)((k >> 1) & 1));
 }
 
 // The same arithmetic with W warps per row (W = 1, 2 or 4) and 8 / W rows per 256-thread
