@@ -303,7 +303,8 @@ size_t bitnet_attention_workspace_bytes(int64_t T, int64_t Hq, int64_t Hkv, int6
 /* Causal grouped-query attention of T new tokens (positions pos0 .. pos0 + T - 1, already in
  * the cache) against cache rows 0 .. pos0 + t: out[t, h] = softmax(q_rot[t, h] . k / sqrt(d)) v
  * with key/value head h / (Hq / Hkv), in fp32 (split over 64-row chunks of the cache, merged
- * exactly as running maxima and sums), written as bf16 or fp32 [T, Hq, d].  T * Hq / Hkv <= 128.
+ * exactly as running maxima and sums), written as bf16 or fp32 [T, Hq, d].  T * Hq / Hkv <= 128,
+ * pos0 + T <= 65536 (SHAPE otherwise).
  * ws: bitnet_attention_workspace_bytes(T, Hq, Hkv, pos0 + T) bytes, 16-byte aligned.
  * Errors: NULL, SHAPE, ALIGN, DTYPE, WORKSPACE. */
 bitnet_status bitnet_attention_decode(const float* q_rot, const void* k_cache, const void* v_cache, int64_t T,

@@ -147,15 +147,17 @@ __global__ void __launch_bounds__(ATT_THREADS) k_attn_partial(const float* __res
     const float* kr = Ks + p * ATT_KP;
     for (int j = rg; j < R; j += ATT_THREADS / ATT_CHUNK) {
       const float* qr = Qs + j * ATT_KP;
-      float acc = 0.0f;
+      // four independent partial sums (short dependency chains), added at the end
+      float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll 8
       for (int d = 0; d < ATT_D; d += 4) {
         const float4 a = *reinterpret_cast<const float4*>(qr + d), b = *reinterpret_cast<const float4*>(kr + d);
-        acc = __fadd_rn(acc, __fmul_rn(a.x, b.x));
-        acc = __fadd_rn(acc, __fmul_rn(a.y, b.y));
-        acc = __fadd_rn(acc, __fmul_rn(a.z, b.z));
-        acc = __fadd_rn(acc, __fmul_rn(a.w, b.w));
+        a0 = __fadd_rn(a0, __fmul_rn(a.x, b.x));
+        a1 = __fadd_rn(a1, __fmul_rn(a.y, b.y));
+        a2 = __fadd_rn(a2, __fmul_rn(a.z, b.z));
+        a3 = __fadd_rn(a3, __fmul_rn(a.w, b.w));
       }
+      const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
       const long long qpos = pos0 + j / G;
       Ss[j * ATT_CHUNK + p] = (p < n && c0 + p <= qpos) ? __fmul_rn(acc, scale) : -INFINITY;
     }
@@ -189,8 +191,16 @@ __global__ void __launch_bounds__(ATT_THREADS) k_attn_partial(const float* __res
     const int d = tid % ATT_D, rh = tid / ATT_D;
     for (int j = rh; j < R; j += ATT_THREADS / ATT_D) {
       const float* sr = Ss + j * ATT_CHUNK;
-      float acc = 0.0f;
-      for (int p = 0; p < n; ++p) acc = __fadd_rn(acc, __fmul_rn(sr[p], Vs[p * ATT_KP + d]));
+      float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+      int p = 0;
+      for (; p + 3 < n; p += 4) {
+        a0 = __fadd_rn(a0, __fmul_rn(sr[p], Vs[p * ATT_KP + d]));
+        a1 = __fadd_rn(a1, __fmul_rn(sr[p + 1], Vs[(p + 1) * ATT_KP + d]));
+        a2 = __fadd_rn(a2, __fmul_rn(sr[p + 2], Vs[(p + 2) * ATT_KP + d]));
+        a3 = __fadd_rn(a3, __fmul_rn(sr[p + 3], Vs[(p + 3) * ATT_KP + d]));
+      }
+      for (; p < n; ++p) a0 = __fadd_rn(a0, __fmul_rn(sr[p], Vs[p * ATT_KP + d]));
+      const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
       float* dst = part + (((long long)chunk * Hkv + kv) * R + j) * (ATT_D + 2);
       dst[d] = acc;
       if (d == 0) {
@@ -202,25 +212,54 @@ __global__ void __launch_bounds__(ATT_THREADS) k_attn_partial(const float* __res
 }
 
 // Merge the chunks of each query row: out = (sum_c o_c e^(m_c - M)) / (sum_c l_c e^(m_c - M)).
+// The chunk maxima and factors go through shared memory (each loaded once, all chunks at once
+// across the 128 threads); every thread then sums its dimension over the chunks with eight
+// loads in flight, so the merge costs a few memory round trips instead of one per chunk.
+constexpr int ATT_MAX_CHUNKS = 1024;  // cache rows up to 64 Ki
 __global__ void __launch_bounds__(ATT_D) k_attn_combine(const float* __restrict__ part, int T, int Hq, int Hkv,
                                                         int n_chunks, void* __restrict__ out, int out_dtype) {
+  __shared__ float s_f[ATT_MAX_CHUNKS];
+  __shared__ float s_red[ATT_D / 32];
   pdl_launch_dependents();
   pdl_wait();
   const int G = Hq / Hkv, R = T * G;
   const int row = blockIdx.x;  // (t, h)
   const int t = row / Hq, h = row % Hq, kv = h / G, j = t * G + (h % G);
-  const int d = threadIdx.x;
+  const int d = threadIdx.x, lane = d & 31, w = d >> 5;
+  auto pc = [&](int c) { return part + (((long long)c * Hkv + kv) * R + j) * (ATT_D + 2); };
   float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, part[(((long long)c * Hkv + kv) * R + j) * (ATT_D + 2) + ATT_D]);
-  float L = 0.0f, O = 0.0f;
-  for (int c = 0; c < n_chunks; ++c) {
-    const float* pc = part + (((long long)c * Hkv + kv) * R + j) * (ATT_D + 2);
-    const float m = pc[ATT_D];
-    if (m == -INFINITY) continue;
-    const float f = expf(__fsub_rn(m, M));
-    L = __fadd_rn(L, __fmul_rn(pc[ATT_D + 1], f));
-    O = __fadd_rn(O, __fmul_rn(pc[d], f));
+  for (int c = d; c < n_chunks; c += ATT_D) {
+    const float m = pc(c)[ATT_D];
+    s_f[c] = m;
+    M = fmaxf(M, m);
   }
+  M = warp_max(M);
+  if (lane == 0) s_red[w] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  __syncthreads();
+  float L = 0.0f;
+  for (int c = d; c < n_chunks; c += ATT_D) {
+    const float m = s_f[c];
+    const float f = m == -INFINITY ? 0.0f : expf(__fsub_rn(m, M));
+    s_f[c] = f;
+    L = __fadd_rn(L, __fmul_rn(pc(c)[ATT_D + 1], f));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L = __fadd_rn(L, __shfl_xor_sync(0xffffffffu, L, o));
+  if (lane == 0) s_red[w] = L;
+  __syncthreads();
+  L = __fadd_rn(__fadd_rn(s_red[0], s_red[1]), __fadd_rn(s_red[2], s_red[3]));
+  float O = 0.0f;
+  int c = 0;
+  for (; c + 7 < n_chunks; c += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = pc(c + k)[d];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) O = __fadd_rn(O, __fmul_rn(v[k], s_f[c + k]));
+  }
+  for (; c < n_chunks; ++c) O = __fadd_rn(O, __fmul_rn(pc(c)[d], s_f[c]));
   store_out(out, out_dtype, (long long)row * ATT_D + d, __fdiv_rn(O, L));
 }
 

@@ -797,7 +797,7 @@ bitnet_status bitnet_attention_decode(const float* q_rot, const void* k_cache, c
                                       bitnet_dtype ot, void* ws, size_t ws_bytes, bitnet_stream stream) {
   if (ot != BITNET_BF16 && ot != BITNET_F32) return BITNET_ERR_DTYPE;
   if (T < 0 || d != ATT_D || Hq <= 0 || Hkv <= 0 || Hq % Hkv || pos0 < 0 || L_max <= 0 || pos0 + T > L_max ||
-      T * (Hq / Hkv) > ATT_MAX_ROWS || Hq > 4096 || (pos0 + T + ATT_CHUNK - 1) / ATT_CHUNK > 65535)
+      T * (Hq / Hkv) > ATT_MAX_ROWS || Hq > 4096 || (pos0 + T + ATT_CHUNK - 1) / ATT_CHUNK > ATT_MAX_CHUNKS)
     return BITNET_ERR_SHAPE;
   if (T == 0) return BITNET_OK;
   if (!q_rot || !k_cache || !v_cache || !out) return BITNET_ERR_NULL;
