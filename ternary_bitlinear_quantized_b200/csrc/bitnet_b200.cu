@@ -850,10 +850,12 @@ bitnet_status bitnet_ffn_workspace_offsets(int64_t T, int64_t H, int64_t I, size
 
 // Per-CTA partial reductions of the distributed sub-norm after the counters (G = ENG_MAX_GRID):
 // max |h| [T][G] fp32, max |y| [T][G] fp32, candidate fixed-point sums [T][G][ENG_SUB_CAND]
-// int64, fallback sums [T][G] int64.
+// int64, fallback sums [T][G] int64, max |y| candidates [T][G] (h, g) fp32 pairs and their counts
+// [T][G] int32.
 static size_t ffn_partials_bytes(int64_t T) {
   return 2 * align_up((size_t)T * ENG_MAX_GRID * 4) + align_up((size_t)T * ENG_MAX_GRID * ENG_SUB_CAND * 8) +
-         (size_t)T * ENG_MAX_GRID * 8;
+         2 * align_up((size_t)T * ENG_MAX_GRID * 8) +
+         (size_t)T * ENG_MAX_GRID * 4;
 }
 
 size_t bitnet_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I) {
@@ -907,6 +909,9 @@ static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32,
     long long* psum = reinterpret_cast<long long*>(pb + 2 * align_up((size_t)T * ENG_MAX_GRID * 4));
     long long* psum_fb = reinterpret_cast<long long*>(pb + 2 * align_up((size_t)T * ENG_MAX_GRID * 4) +
                                                       align_up((size_t)T * ENG_MAX_GRID * ENG_SUB_CAND * 8));
+    uint8_t* pyb = reinterpret_cast<uint8_t*>(psum_fb) + align_up((size_t)T * ENG_MAX_GRID * 8);
+    float2* pyc = reinterpret_cast<float2*>(pyb);
+    int* pycnt = reinterpret_cast<int*>(pyb + align_up((size_t)T * ENG_MAX_GRID * 8));
     gate_up.pmax = pmax;
     gate_up.sub_gain = g_sub;
     ea.ph[ea.n_phases++] = gate_up;
@@ -925,6 +930,8 @@ static void plan_ffn(EngArgs& ea, int& bar, int wait0, const void* x, int x_f32,
     sp.pmax2 = pmax2;
     sp.psum = psum;
     sp.psum_fb = psum_fb;
+    sp.pyc = pyc;
+    sp.pycnt = pycnt;
     sp.wait_barrier = -1;
     sp.bar_a = bar++;
     sp.bar_b = bar++;

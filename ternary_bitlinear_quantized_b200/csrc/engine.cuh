@@ -88,6 +88,8 @@ struct EngPhase {
   long long* psum;
   long long* psum_fb;
   float* pmax2;
+  float2* pyc;  // per CTA and token: the (h, g) pair that may hold max |y| [T][G]
+  int* pycnt;   // the count of such pairs [T][G] (2: more than one)
   const float* sub_gain;
   int bar_a, bar_b, bar_fb;
   // Tile split over the grid: CTA c owns tiles [start(c), start(c + 1)); by default
@@ -414,6 +416,10 @@ BN_DEV bool grid_wait(unsigned* ctr, unsigned target) {
 constexpr int ENG_SUB_CAND = 8;  // candidate grids per CTA: local exponent e_c, e_c - 1, .., e_c - 7
 static_assert(ENG_SUB_CAND == 8, "the candidate sums are reduced by a three-level lane split");
 struct SubScratch {
+  unsigned long long pmx[ENG_MAX_T];  // this CTA's max |h g| (exact, fp64 bits; non-negative)
+  float2 yc[ENG_MAX_T];               // an (h, g) pair within 2^-20 of it
+  int ycnt[ENG_MAX_T];                // and how many there are
+  int yfb;                            // some CTA had more than one candidate: the barrier path
   unsigned mx[ENG_MAX_T];  // max |h|: this CTA's, then the row's (non-negative floats as bits)
   unsigned my[ENG_MAX_T];  // max |y|
   unsigned long long sum[ENG_MAX_T];
@@ -444,7 +450,9 @@ BN_DEV bool grid_step(unsigned* ctr) {
 //      e (or M_c = 0, whose sum is 0 on any grid) the sum is the sum of those candidates,
 //      else (uniformly, from the same published maxima) every CTA sums on e itself and a
 //      second barrier publishes those sums;
-//   3. inv, max |y| of the CTA's rows -> published; grid barrier; 4. s_x and q of its rows.
+//   3. inv, and max |y| from the (h, g) candidate each CTA published with its sums; when
+//      some CTA had more than one candidate (or after the sum fallback), max |y| of every
+//      CTA's rows -> published; grid barrier; 4. s_x and q of its rows.
 // Maxima and integer sums are order-free, so the result does not depend on the split.
 // p.sq must be zero on entry (the kernel clears it before the gate/up phase).
 __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, int tb, int te, unsigned* counters,
@@ -458,16 +466,31 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
   if (tid < T) {
     S.mx[tid] = S.my[tid] = 0u;
     S.sum[tid] = 0ull;
+    S.pmx[tid] = 0ull;
+    S.ycnt[tid] = 0;
 #pragma unroll
     for (int d = 0; d < ENG_SUB_CAND; ++d) S.cand[tid][d] = 0ull;
   }
-  if (tid == 0) S.fallback = 0;
+  if (tid == 0) S.fallback = S.yfb = 0;
   cons_sync();
-  // 1. this CTA's max |h|, then its sums on the candidate grids e_c - d
+  // 1. this CTA's max |h| and max |h g| (exact in fp64), then its sums on the candidate grids
+  // e_c - d, and the (h, g) pair whose |h g| is within 2^-20 of the CTA's maximum (with the
+  // count of such pairs).  max |y| over the row is taken at one of those: y = fl(fl(h inv) g)
+  // is |h g| inv within a relative 2^-23 (for the y that can set the scale: |y| >= 1e-5 and
+  // gains far below 2^100), so an element whose |h g| is below the row's maximum by more than
+  // 2^-22 cannot hold it, and the row's argmax lies within 2^-22 of its own CTA's maximum.
   for (int it = warp; it < items; it += ENG_CONS_WARPS) {
     const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
-    const float m = warp_max(r < nrows ? fabsf(hs[t * sub_rows + r]) : 0.0f);
+    const float hv = r < nrows ? hs[t * sub_rows + r] : 0.0f;
+    const float m = warp_max(fabsf(hv));
     if (lane == 0) atomicMax(&S.mx[t], __float_as_uint(m));
+    if (p.gain != nullptr) {
+      const double pr = r < nrows ? fabs(__dmul_rn((double)hv, (double)gs[r])) : 0.0;
+      unsigned long long pb = (unsigned long long)__double_as_longlong(pr);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) pb = max(pb, __shfl_xor_sync(0xffffffffu, pb, o));
+      if (lane == 0) atomicMax(&S.pmx[t], pb);
+    }
   }
   cons_sync();
   if (tid < T) {
@@ -480,6 +503,14 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
       if (S.mx[t] == 0u) continue;
       const float v = r < nrows ? hs[t * sub_rows + r] : 0.0f;
+      // the max |y| candidate of this row
+      const double pc = __longlong_as_double((long long)S.pmx[t]);
+      if (pc > 0.0 && r < nrows) {
+        const float gv = gs[r];
+        if (fabs(__dmul_rn((double)v, (double)gv)) >= __dsub_rn(pc, __dmul_rn(pc, 0x1p-20))) {
+          if (atomicAdd(&S.ycnt[t], 1) == 0) S.yc[t] = make_float2(v, gv);
+        }
+      }
       const double d2 = __dmul_rn((double)v, (double)v);
       double p2e = pow2_f64(S.e[t]);
       long long c[ENG_SUB_CAND];
@@ -518,20 +549,31 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     if (tid < T * ENG_SUB_CAND)
       p.psum[((long long)(tid / ENG_SUB_CAND) * G + blockIdx.x) * ENG_SUB_CAND + tid % ENG_SUB_CAND] =
           (long long)S.cand[tid / ENG_SUB_CAND][tid % ENG_SUB_CAND];
+    if (tid < T) {
+      p.pyc[tid * G + blockIdx.x] = S.yc[tid];
+      p.pycnt[tid * G + blockIdx.x] = min(S.ycnt[tid], 2);
+    }
   }
   if (tid < T) p.pmax[tid * G + blockIdx.x] = __uint_as_float(S.mx[tid]);
   if (!grid_step(counters + p.bar_a)) return false;
-  // 2. the global max; the sum from the candidates when they cover the global grid.  A warp
-  // per token loads the G published maxima at once (unrolled, predicated: one round trip),
-  // reduces them with shuffles, then loads the matching candidate sums at once (a second
-  // round trip).  No shared-memory atomics on one address.
+  // 2. + 3. A warp per token loads every CTA's published max |h|, candidate count and (h, g)
+  // pair at once (one round trip), reduces the max with shuffles, then loads the matching
+  // candidate sums (a second round trip): the row's exact sum of squares, inv, and max |y| from
+  // the candidates -- the same values in every CTA.  Two uniform exceptions take the barrier
+  // path: a CTA whose candidate grids miss the row's grid (the sum is taken again on the row's
+  // grid), or one with more than one max |y| candidate (max |y| over every CTA's rows).
   constexpr int GPL = ENG_MAX_GRID / 32;  // published values per lane at most
   for (int t = warp; t < T; t += ENG_CONS_WARPS) {
     float pm[GPL];
+    int cn[GPL];
+    float2 hg[GPL];
 #pragma unroll
     for (int j = 0; j < GPL; ++j) {
       const int c = lane + 32 * j;
-      pm[j] = c < G ? __ldcg(p.pmax + t * G + c) : 0.0f;
+      const bool in = c < G;
+      pm[j] = in ? __ldcg(p.pmax + t * G + c) : 0.0f;
+      cn[j] = (in && p.gain != nullptr) ? __ldcg(p.pycnt + t * G + c) : 0;
+      hg[j] = (in && p.gain != nullptr) ? __ldcg(p.pyc + t * G + c) : make_float2(0.0f, 0.0f);
     }
     float m = 0.0f;
 #pragma unroll
@@ -540,10 +582,11 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
     const int e = m > 0.0f ? fixed_point_exponent(__dmul_rn((double)m, (double)m), K) : 0;
     if (p.gain != nullptr) {
       long long v[GPL];
-      int fb = 0;
+      int fb = 0, over = 0;
 #pragma unroll
       for (int j = 0; j < GPL; ++j) {
         v[j] = 0;
+        if (cn[j] > 1) over = 1;
         if (pm[j] > 0.0f) {
           const int d = fixed_point_exponent(__dmul_rn((double)pm[j], (double)pm[j]), K) - e;
           if (d >= ENG_SUB_CAND)
@@ -557,9 +600,22 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       for (int j = 0; j < GPL; ++j) sum += v[j];
       sum = warp_sum_ll(sum);
       fb = __any_sync(0xffffffffu, fb);
+      over = __any_sync(0xffffffffu, over);
+      float ymax = 0.0f, inv = 0.0f;
+      if (!fb && !over) {
+        const float ms = m > 0.0f ? fixed_point_mean(sum, e, K) : 0.0f;
+        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+#pragma unroll
+        for (int j = 0; j < GPL; ++j)
+          if (cn[j] == 1) ymax = fmaxf(ymax, fabsf(__fmul_rn(__fmul_rn(hg[j].x, inv), hg[j].y)));
+        ymax = warp_max(ymax);
+      }
       if (lane == 0) {
         S.sum[t] = (unsigned long long)sum;
         if (fb) S.fallback = 1;
+        if (over) S.yfb = 1;
+        S.inv[t] = inv;
+        S.my[t] = __float_as_uint(ymax);
       }
     }
     if (lane == 0) {
@@ -589,36 +645,38 @@ __device__ __noinline__ bool eng_subnorm(const EngPhase& p, int T, float eps, in
       }
       cons_sync();
     }
-    // 3. inv and max |y| of this CTA's rows
-    if (tid < T) {
-      const float am = __uint_as_float(S.mx[tid]);
-      const float ms = am > 0.0f ? fixed_point_mean((long long)S.sum[tid], S.e[tid], K) : 0.0f;
-      S.inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-    }
-    cons_sync();
-    for (int it = warp; it < items; it += ENG_CONS_WARPS) {
-      const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
-      const float y = r < nrows ? fabsf(__fmul_rn(__fmul_rn(hs[t * sub_rows + r], S.inv[t]), gs[r])) : 0.0f;
-      const float m = warp_max(y);
-      if (lane == 0) atomicMax(&S.my[t], __float_as_uint(m));
-    }
-    cons_sync();
-    if (tid < T) p.pmax2[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
-    if (!grid_step(counters + p.bar_b)) return false;
-    for (int t = warp; t < T; t += ENG_CONS_WARPS) {
-      float pm[GPL];
-#pragma unroll
-      for (int j = 0; j < GPL; ++j) {
-        const int c = lane + 32 * j;
-        pm[j] = c < G ? __ldcg(p.pmax2 + t * G + c) : 0.0f;
+    if (S.fallback || S.yfb) {  // uniform: max |y| over this CTA's rows and a grid barrier
+      if (tid < T) {
+        const float am = __uint_as_float(S.mx[tid]);
+        const float ms = am > 0.0f ? fixed_point_mean((long long)S.sum[tid], S.e[tid], K) : 0.0f;
+        S.inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+        S.my[tid] = 0u;
       }
-      float m = 0.0f;
+      cons_sync();
+      for (int it = warp; it < items; it += ENG_CONS_WARPS) {
+        const int t = it / chunks, r = (it - t * chunks) * 32 + lane;
+        const float y = r < nrows ? fabsf(__fmul_rn(__fmul_rn(hs[t * sub_rows + r], S.inv[t]), gs[r])) : 0.0f;
+        const float mm = warp_max(y);
+        if (lane == 0) atomicMax(&S.my[t], __float_as_uint(mm));
+      }
+      cons_sync();
+      if (tid < T) p.pmax2[tid * G + blockIdx.x] = __uint_as_float(S.my[tid]);
+      if (!grid_step(counters + p.bar_b)) return false;
+      for (int t = warp; t < T; t += ENG_CONS_WARPS) {
+        float pm[GPL];
 #pragma unroll
-      for (int j = 0; j < GPL; ++j) m = fmaxf(m, pm[j]);
-      m = warp_max(m);
-      if (lane == 0) S.my[t] = __float_as_uint(m);
+        for (int j = 0; j < GPL; ++j) {
+          const int c = lane + 32 * j;
+          pm[j] = c < G ? __ldcg(p.pmax2 + t * G + c) : 0.0f;
+        }
+        float mm = 0.0f;
+#pragma unroll
+        for (int j = 0; j < GPL; ++j) mm = fmaxf(mm, pm[j]);
+        mm = warp_max(mm);
+        if (lane == 0) S.my[t] = __float_as_uint(mm);
+      }
+      cons_sync();
     }
-    cons_sync();
   } else {
     if (tid < T) {
       S.my[tid] = S.mx[tid];  // y = h

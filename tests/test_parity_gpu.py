@@ -319,6 +319,36 @@ def test_ffn_block_distributed_sub_norm_fallback(T):
     assert tb.device_status() == 0
 
 
+@pytest.mark.parametrize("T", [1, 3])
+def test_ffn_block_distributed_sub_norm_ymax_ties(T):
+    """max |y| of the grid-wide ffn_sub_norm comes from each CTA's published (h, g) pairs near
+    its max |h g| unless a CTA has more such pairs than it can publish; here every gate row
+    and every up row is the same and the sub-norm gain is constant, so |h g| ties on every row
+    and the grid-barrier path runs; bit-exact either way."""
+    H, I = 512, 16512
+    sh = workloads.BlockShape("ffn-ties", hidden=H, n_q=H, n_kv=H, inter=I, act="relu2")
+    d = workloads.block_inputs(sh, T, 78, ffn_only=True)
+    Wg = d["W_gate"][:1].repeat(I, 1).contiguous()
+    Wu = d["W_up"][:1].repeat(I, 1).contiguous()
+    g_sub = torch.full_like(d["g_ffn_sub_norm"], 1.5)
+    pr = {"gate": O.pack_i2s(Wg.numpy()), "up": O.pack_i2s(Wu.numpy()), "down": O.pack_i2s(d["W_down"].numpy())}
+    pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
+    ws = torch.zeros(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
+    ref, mid = O.ffn_block(bf16_to_np(d["x"]), d["g_ffn_norm"].numpy(), pr["gate"], pr["up"], g_sub.numpy(),
+                           pr["down"], H, I, "relu2", 1e-6, "bf16", return_intermediates=True)
+    assert np.all(mid["h"] == mid["h"][:, :1])  # every row of h the same
+    off = tb.ffn_workspace_offsets(T, H, I)
+    for _ in range(2):
+        out = tb.ffn_block(d["x"].to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], g_sub.to(DEV),
+                           pg["down"], I, tb.RELU2, 1e-6, torch.bfloat16, ws=ws)
+        torch.cuda.synchronize()
+        wsn = ws.cpu().numpy()
+        assert np.array_equal(wsn[off[4]:off[4] + T * I].view(np.int8).reshape(T, I), mid["q_h"])
+        assert np.array_equal(wsn[off[6]:off[6] + T * 4].view(np.int32), mid["sum_h"])
+        assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
+    assert tb.device_status() == 0
+
+
 def test_ffn_block_fp32_io():
     out, _, ref, _, dt = run_ffn(2, 384, 512, "silu", seed=5, out_dtype=torch.float32, x_dtype=torch.float32)
     assert np.array_equal(out_to_np(out).view(np.uint32), ref.view(np.uint32))
