@@ -144,7 +144,7 @@ static bitnet_status enqueue_quant(const void* x, bitnet_dtype xt, const float* 
     return BITNET_OK;
   }
   // Long fp32 rows, many of them (the FFN's h at prefill): persistent, double-buffered.
-  if (xt == BITNET_F32 && K % 4 == 0 && 2 * K * 4 <= 227 * 1024 - 1024 && K <= QL_THREADS * QL_MAXJ &&
+  if (xt == BITNET_F32 && K % 4 == 0 && 2 * K * 4 <= 227 * 1024 - 1024 && K <= 4 * QL_THREADS * QL_MAXV &&
       T >= 2 * device_sm_count() && aligned16(x) && aligned16(q)) {
     const size_t smem_l = (size_t)2 * K * 4;
     static std::atomic<int> long_done[64] = {};

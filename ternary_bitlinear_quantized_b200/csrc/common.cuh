@@ -260,19 +260,40 @@ BN_DEV T block_reduce(T v, T* scratch, Op op) {
   __syncthreads();  // scratch may still be read by a previous reduction
   if (lane == 0) scratch[warp] = v;
   __syncthreads();
-  T r = scratch[0];
-  for (int w = 1; w < nw; ++w) r = op(r, scratch[w]);
+  // every warp reduces the (at most 32) warp results with shuffles: one shared load per thread
+  T r = lane < nw ? scratch[lane] : Op::identity();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) r = op(r, __shfl_xor_sync(0xffffffffu, r, o));
+  return r;
+}
+
+// The same with one barrier instead of two: consecutive calls alternate between two scratch
+// areas, so a call's area is rewritten only after the following call's barrier, which every
+// thread reaches after it has read that area.
+template <typename T, typename Op>
+BN_DEV T block_reduce_alt(T v, T* scratch, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  T r = lane < nw ? scratch[lane] : Op::identity();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) r = op(r, __shfl_xor_sync(0xffffffffu, r, o));
   return r;
 }
 
 struct MaxOp {
   BN_DEV float operator()(float a, float b) const { return fmaxf(a, b); }
+  BN_DEV static float identity() { return -INFINITY; }
 };
 struct AddOpLL {
   BN_DEV long long operator()(long long a, long long b) const { return a + b; }
+  BN_DEV static long long identity() { return 0; }
 };
 struct AddOpI {
   BN_DEV int operator()(int a, int b) const { return a + b; }
+  BN_DEV static int identity() { return 0; }
 };
 
 }  // namespace bitnet

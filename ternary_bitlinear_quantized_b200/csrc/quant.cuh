@@ -152,30 +152,37 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_quant(const TIn* __restrict__ 
 }
 
 // Long fp32 rows (the FFN's h at prefill): one CTA per SM, persistent over rows blockIdx.x,
-// blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with one
-// bulk copy (completing on the buffer's mbarrier) while the current one is reduced, so the
-// row reads stream at the HBM rate instead of waiting behind each row's reduction chain.  Thread i owns elements
-// i + QL_THREADS j; its gain values stay in registers for all rows (reading them from L2 per
-// row put a memory round trip behind every element of the y pass).  The arithmetic is
-// quantise_staged_row's.  K % 4 == 0, K <= QL_THREADS QL_MAXJ, rows 16-byte aligned,
+// blockIdx.x + gridDim.x, ...; two row buffers in shared memory, the next row fetched with a
+// set of bulk copies (completing on the buffer's mbarrier) while the current one is reduced,
+// so the row reads stream at the HBM rate instead of waiting behind each row's reduction
+// chain.  Thread i owns the four elements 4 (i + QL_THREADS j) .. + 3 of every group j, read
+// from shared memory with 16-byte loads; its gain values stay in registers for all rows
+// (reading them from L2 per row put a memory round trip behind every element of the y pass).
+// The y pass writes y over the row; the q pass writes four codes per 4-byte store.  The
+// reductions use one barrier each and are the row's only barriers.  The arithmetic is
+// quantise_staged_row's.  K % 4 == 0, K <= 4 QL_THREADS QL_MAXV, rows 16-byte aligned,
 // 2 K floats of shared memory.
 constexpr int QL_THREADS = 1024;
-constexpr int QL_MAXJ = 28;  // K <= 28672
+constexpr int QL_MAXV = 7;  // K <= 28672
+constexpr int QL_PARTS = 8;  // bulk copies per row
 __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const float* __restrict__ x,
                                                                      const float* __restrict__ gain, float eps,
                                                                      int T, int K, int8_t* __restrict__ q,
                                                                      float* __restrict__ s_x,
                                                                      int32_t* __restrict__ sum_q) {
   extern __shared__ __align__(16) float ql_buf[];  // [2][K]
-  __shared__ long long red[32];
+  __shared__ long long red[2][32];  // the two scratch areas of the reductions, used in turn
+  int ra = 0;
   __shared__ __align__(8) unsigned long long ql_bar[2];  // one per row buffer: its bulk copy landed
   volatile __shared__ int ql_abort;
   const int tid = threadIdx.x;
-  float gr[QL_MAXJ];
+  const int K4 = K >> 2;
+  float4 gr[QL_MAXV];
 #pragma unroll
-  for (int j = 0; j < QL_MAXJ; ++j) {
-    const int k = tid + QL_THREADS * j;
-    gr[j] = (gain != nullptr && k < K) ? __ldg(gain + k) : 0.0f;
+  for (int j = 0; j < QL_MAXV; ++j) {
+    const int k4 = tid + QL_THREADS * j;
+    gr[j] = (gain != nullptr && k4 < K4) ? __ldg(reinterpret_cast<const float4*>(gain) + k4)
+                                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
   if (tid == 0) {
     mbar_init(smem_addr(&ql_bar[0]), 1);
@@ -186,11 +193,15 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
   __syncthreads();
   pdl_launch_dependents();
   pdl_wait();
-  // One bulk copy per row (thread 0), completing on the buffer's barrier.
+  // A row is fetched by thread 0 as QL_PARTS bulk copies (several in flight stream faster than
+  // one long copy), all completing on the buffer's barrier.
   const uint32_t row_bytes = (uint32_t)K * 4u;
+  const uint32_t part = (row_bytes + 16u * QL_PARTS - 1u) / (16u * QL_PARTS) * 16u;  // multiple of 16
   auto fetch = [&](long long row, int b) {
-    mbar_arrive_expect_tx(smem_addr(&ql_bar[b]), row_bytes);
-    bulk_g2s(smem_addr(ql_buf + b * K), x + row * K, row_bytes, smem_addr(&ql_bar[b]));
+    const uint32_t bar = smem_addr(&ql_bar[b]), dst = smem_addr(ql_buf + b * K);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(x + row * K);
+    mbar_arrive_expect_tx(bar, row_bytes);
+    for (uint32_t o = 0; o < row_bytes; o += part) bulk_g2s(dst + o, src + o, min(part, row_bytes - o), bar);
   };
   long long row = blockIdx.x;
   int issued = 0;
@@ -200,23 +211,27 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
   }
   for (int it = 0; row < T; ++it, row += gridDim.x) {
     const int b = it & 1;
-    float* cur = ql_buf + b * K;
+    float4* cur = reinterpret_cast<float4*>(ql_buf + b * K);
     const long long next = row + gridDim.x;
-    if (tid == 0 && next < T) {  // the other buffer was released by the barrier at the end of it - 1
+    if (tid == 0 && next < T) {  // the other buffer was released by the last barrier of it - 1
       fetch(next, b ^ 1);
       ++issued;
     }
+    // A wait that gives up is seen by every thread after the first reduction's barrier (the
+    // max pass before it may read an incomplete row; its result is not used).
     if (!mbar_wait_bounded(smem_addr(&ql_bar[b]), (uint32_t)((it >> 1) & 1))) ql_abort = 1;
-    __syncthreads();
-    if (ql_abort) break;
     float am = 0.0f;
 #pragma unroll
-    for (int j = 0; j < QL_MAXJ; ++j) {
-      const int k = tid + QL_THREADS * j;
-      if (k < K) am = fmaxf(am, fabsf(cur[k]));
+    for (int j = 0; j < QL_MAXV; ++j) {
+      const int k4 = tid + QL_THREADS * j;
+      if (k4 < K4) {
+        const float4 v = cur[k4];
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
     }
-    am = block_reduce(am, reinterpret_cast<float*>(red), MaxOp());
-    float a = am;
+    am = block_reduce_alt(am, reinterpret_cast<float*>(red[ra++ & 1]), MaxOp());
+    if (ql_abort) break;
+    float a = am, inv = 1.0f;
     if (gain != nullptr) {
       float ms = 0.0f;
       if (am > 0.0f) {
@@ -224,52 +239,91 @@ __global__ void __launch_bounds__(QL_THREADS, 1) k_rmsnorm_quant_long(const floa
         const double p2e = pow2_f64(e);
         long long part = 0;
         if (K >= kFixedSmallMinN) {
+          // Each term rint(v^2 2^e) < 2^51 as the bits of the fp64 sum 1.5 * 2^52 + v^2 2^e:
+          // v (v 2^e) is exact (a power-of-two scaling, or below 2^-1022 where the term is 0
+          // either way), so one fused multiply-add rounds exactly once, like the rounding add
+          // of fixed_sq_term_t.  The bits are summed as they are (mod 2^64) and the offset of
+          // every term taken off once.
+          unsigned long long bits = 0ull;
+          int n = 0;
 #pragma unroll
-          for (int j = 0; j < QL_MAXJ; ++j) {
-            const int k = tid + QL_THREADS * j;
-            if (k < K) part += fixed_sq_term_t<true>(cur[k], p2e);
+          for (int j = 0; j < QL_MAXV; ++j) {
+            const int k4 = tid + QL_THREADS * j;
+            if (k4 < K4) {
+              const float4 v = cur[k4];
+              const double d0 = (double)v.x, d1 = (double)v.y, d2 = (double)v.z, d3 = (double)v.w;
+              constexpr double kRound = 6755399441055744.0;  // 1.5 * 2^52
+              bits += (unsigned long long)__double_as_longlong(__fma_rn(d0, __dmul_rn(d0, p2e), kRound)) +
+                      (unsigned long long)__double_as_longlong(__fma_rn(d1, __dmul_rn(d1, p2e), kRound)) +
+                      (unsigned long long)__double_as_longlong(__fma_rn(d2, __dmul_rn(d2, p2e), kRound)) +
+                      (unsigned long long)__double_as_longlong(__fma_rn(d3, __dmul_rn(d3, p2e), kRound));
+              n += 4;
+            }
           }
+          part = (long long)(bits - (unsigned long long)n * 0x4338000000000000ull);
         } else {
 #pragma unroll
-          for (int j = 0; j < QL_MAXJ; ++j) {
-            const int k = tid + QL_THREADS * j;
-            if (k < K) part += fixed_sq_term(cur[k], p2e);
+          for (int j = 0; j < QL_MAXV; ++j) {
+            const int k4 = tid + QL_THREADS * j;
+            if (k4 < K4) {
+              const float4 v = cur[k4];
+              part += fixed_sq_term(v.x, p2e) + fixed_sq_term(v.y, p2e) + fixed_sq_term(v.z, p2e) +
+                      fixed_sq_term(v.w, p2e);
+            }
           }
         }
-        ms = fixed_point_mean(block_reduce(part, red, AddOpLL()), e, K);
+        ms = fixed_point_mean(block_reduce_alt(part, red[ra++ & 1], AddOpLL()), e, K);
       }
-      const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+      inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
       float ay = 0.0f;
 #pragma unroll
-      for (int j = 0; j < QL_MAXJ; ++j) {
-        const int k = tid + QL_THREADS * j;
-        if (k < K) {
-          const float y = __fmul_rn(__fmul_rn(cur[k], inv), gr[j]);
-          cur[k] = y;
-          ay = fmaxf(ay, fabsf(y));
+      for (int j = 0; j < QL_MAXV; ++j) {
+        const int k4 = tid + QL_THREADS * j;
+        if (k4 < K4) {
+          float4 v = cur[k4];
+          v.x = __fmul_rn(__fmul_rn(v.x, inv), gr[j].x);
+          v.y = __fmul_rn(__fmul_rn(v.y, inv), gr[j].y);
+          v.z = __fmul_rn(__fmul_rn(v.z, inv), gr[j].z);
+          v.w = __fmul_rn(__fmul_rn(v.w, inv), gr[j].w);
+          ay = fmaxf(ay, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+          cur[k4] = v;  // y, read by the q pass
         }
       }
-      a = block_reduce(ay, reinterpret_cast<float*>(red), MaxOp());
+      fence_proxy_async_smem();  // this thread's y writes ordered before the buffer's next bulk copy
+      a = block_reduce_alt(ay, reinterpret_cast<float*>(red[ra++ & 1]), MaxOp());
     }
     const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
-    int sum = 0;
-    int8_t* qrow = q + row * K;
+    // quant_code's steps with its offset kept: the fp32 bits of clamp(p) + 1.5 * 2^23 are
+    // 0x4B400000 + code, so their low byte is the code's byte; the bits are summed as they are
+    // (mod 2^32) and the offset of every element taken off once.
+    uint32_t cbits = 0u;
+    int n = 0;
+    uint32_t* qrow = reinterpret_cast<uint32_t*>(q + row * K);
 #pragma unroll
-    for (int j = 0; j < QL_MAXJ; ++j) {
-      const int k = tid + QL_THREADS * j;
-      if (k < K) {
-        const int v = quant_code(__fmul_rn(cur[k], s));
-        sum += v;
-        qrow[k] = (int8_t)v;
+    for (int j = 0; j < QL_MAXV; ++j) {
+      const int k4 = tid + QL_THREADS * j;
+      if (k4 < K4) {
+        const float4 y = cur[k4];
+        const float p[4] = {__fmul_rn(y.x, s), __fmul_rn(y.y, s), __fmul_rn(y.z, s), __fmul_rn(y.w, s)};
+        uint32_t b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float c = p[i] == p[i] ? fminf(fmaxf(p[i], -128.0f), 127.0f) : 0.0f;  // NaN: code 0
+          b[i] = __float_as_uint(__fadd_rn(c, 12582912.0f));
+        }
+        cbits += (b[0] + b[1]) + (b[2] + b[3]);
+        n += 4;
+        qrow[k4] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
       }
     }
-    sum = block_reduce(sum, reinterpret_cast<int*>(red), AddOpI());
+    const int sum = block_reduce_alt((int)(cbits - (uint32_t)n * 0x4B400000u), reinterpret_cast<int*>(red[ra++ & 1]),
+                                     AddOpI());
     if (tid == 0) {
       s_x[row] = s;
       sum_q[row] = sum;
     }
-    fence_proxy_async_smem();  // this thread's y writes ordered before the buffer's next bulk copy
-    __syncthreads();           // the buffer is refilled by the fetch of the next iteration
+    // The buffer is refilled by the fetch of iteration it + 1, issued after the barrier of the
+    // reduction above, which every thread reaches after its last read of the buffer.
   }
   // After a wait gave up, the copies still in flight land (fixed limit) before the CTA exits.
   if (tid == 0 && ql_abort)

@@ -117,6 +117,8 @@ def test_validate_i2s_matches_oracle(N, K):
     (130, 384, torch.bfloat16, True, True),
     (300, 27648, torch.float32, True, False),   # long fp32 rows, many of them: persistent double-buffered kernel
     (301, 12288, torch.float32, False, True),
+    (300, 1020, torch.float32, True, True),     # long-row kernel, rows of <= 1024 values: the general sum terms
+    (297, 9000, torch.float32, True, True),     # long-row kernel, K not a multiple of 16
 ])
 def test_quant_bitexact(T, K, dtype, use_gain, outliers):
     x = workloads.activations(T, K, 11, "quant", outliers)
