@@ -321,24 +321,35 @@ def test_ffn_block_distributed_sub_norm_fallback(T):
     assert tb.device_status() == 0
 
 
-@pytest.mark.parametrize("T", [1, 3])
-def test_ffn_block_distributed_sub_norm_ymax_ties(T):
-    """max |y| of the grid-wide ffn_sub_norm comes from each CTA's published (h, g) pairs near
-    its max |h g| unless a CTA has more such pairs than it can publish; here every gate row
-    and every up row is the same and the sub-norm gain is constant, so |h g| ties on every row
-    and the grid-barrier path runs; bit-exact either way."""
+@pytest.mark.parametrize("T,mode", [(1, "all"), (3, "all"), (300, "all"), (300, "tile0")])
+def test_ffn_block_distributed_sub_norm_ymax_ties(T, mode):
+    """max |y| of the decode engine's grid-wide ffn_sub_norm comes from each CTA's (h, g)
+    candidate near its largest |h g| unless a CTA has several; here every gate row and every up
+    row is the same and the sub-norm gain is constant ("all": |h g| ties everywhere), or only the
+    first 128 rows of gate and up and the first 128 gain values are ("tile0"), so the grid-barrier
+    path runs.  T = 300 takes the prefill path (long-row quantisation of h) on the same ties.
+    Bit-exact either way."""
     H, I = 512, 16512
     sh = workloads.BlockShape("ffn-ties", hidden=H, n_q=H, n_kv=H, inter=I, act="relu2")
     d = workloads.block_inputs(sh, T, 78, ffn_only=True)
-    Wg = d["W_gate"][:1].repeat(I, 1).contiguous()
-    Wu = d["W_up"][:1].repeat(I, 1).contiguous()
-    g_sub = torch.full_like(d["g_ffn_sub_norm"], 1.5)
+    if mode == "all":
+        Wg = d["W_gate"][:1].repeat(I, 1).contiguous()
+        Wu = d["W_up"][:1].repeat(I, 1).contiguous()
+        g_sub = torch.full_like(d["g_ffn_sub_norm"], 1.5)
+    else:
+        Wg, Wu, g_sub = d["W_gate"].clone(), d["W_up"].clone(), d["g_ffn_sub_norm"].clone()
+        Wg[:128] = Wg[:1]
+        Wu[:128] = Wu[:1]
+        g_sub[:128] = 1.5
     pr = {"gate": O.pack_i2s(Wg.numpy()), "up": O.pack_i2s(Wu.numpy()), "down": O.pack_i2s(d["W_down"].numpy())}
     pg = {nm: torch.from_numpy(v).to(DEV) for nm, v in pr.items()}
     ws = torch.zeros(tb.ffn_workspace_bytes(T, H, I), dtype=torch.uint8, device=DEV)
     ref, mid = O.ffn_block(bf16_to_np(d["x"]), d["g_ffn_norm"].numpy(), pr["gate"], pr["up"], g_sub.numpy(),
                            pr["down"], H, I, "relu2", 1e-6, "bf16", return_intermediates=True)
-    assert np.all(mid["h"] == mid["h"][:, :1])  # every row of h the same
+    if mode == "all":
+        assert np.all(mid["h"] == mid["h"][:, :1])  # every row of h the same
+    else:
+        assert np.all(mid["h"][:, :128] == mid["h"][:, :1])
     off = tb.ffn_workspace_offsets(T, H, I)
     for _ in range(2):
         out = tb.ffn_block(d["x"].to(DEV), d["g_ffn_norm"].to(DEV), pg["gate"], pg["up"], g_sub.to(DEV),
